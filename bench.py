@@ -1,0 +1,375 @@
+"""Throughput of the Attamba layer forward hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = the whole prefill hot path on one batch of the inference-mask
+workload (B=4, n=4096, d_model=1024, 16 heads x 64, N=16, P=8, L=64, M_test,
+bf16): chunk index -> KV-SSM scan (K and V) -> chunk-masked attention, three
+C-ABI calls on inputs already resident in HBM.  L2 is flushed between steps
+(a 256 MiB write, outside the per-step events).  Each rank runs its own batch
+(weak scaling, no collective on the data path); the time is the max over ranks.
+
+--impl reference times the CPU oracle (float64 numpy, test infrastructure) on
+this host's cores on a bounded sample of the same workload.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from ssm_compressed_chunked_b200 import workloads as W  # noqa: E402
+
+METRIC = "Attamba layer fwd tokens/s at n=4096,P=8,L=64 bf16"
+UNIT = "tokens/s"
+CFG = W.LAYER_CONFIGS[2]
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def config_block(cfg, extra=None):
+    c = {"workload": cfg.name, "batch": cfg.B, "seq_len": cfg.n, "d_model": cfg.D, "heads": cfg.H,
+         "head_dim": cfg.dh, "ssm_state": cfg.N, "chunk": cfg.P, "offset": cfg.offset, "leading_tokens": cfg.L,
+         "mask": "M_" + cfg.mode, "seed": cfg.seed, "l2": "flushed between steps (256 MiB write)"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def source_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, "ssm_compressed_chunked_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged since."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel)
+    if not d or d.get("source_sha") != source_sha(d["sources"]):
+        return None
+    return d["bytes_per_launch_full"]
+
+
+def setup_dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ CPU oracle (reference arm / baseline)
+def oracle_sample(inp, n_tok):
+    """The oracle on sequence 0 truncated to n_tok tokens, all heads: scan K/V + dense M_test attention."""
+    from oracle import attention as OA, chunks as OC, mask as OM, ssm as OS
+    cfg = inp["cfg"]
+    f = lambda t: t.detach().to(torch.float64).numpy()
+    st = OC.uniform_starts(n_tok, cfg.P, cfg.offset)
+    is_start = OC.is_start_mask(st, n_tok)
+    sl = slice(0, n_tok)
+    K, _ = OS.selective_scan(f(inp["x"][0, sl]), f(inp["dt_k"][0, sl]), f(inp["bias_k"]), f(inp["A_k"]),
+                             f(inp["B_k"][0, sl]), f(inp["C_k"][0, sl]), is_start)
+    V, _ = OS.selective_scan(f(inp["x"][0, sl]), f(inp["dt_v"][0, sl]), f(inp["bias_v"]), f(inp["A_v"]),
+                             f(inp["B_v"][0, sl]), f(inp["C_v"][0, sl]), is_start)
+    M = OM.dense_mask(n_tok, st, cfg.L, cfg.mode)
+    OA.masked_attention(f(inp["q"][0, sl]), K.reshape(n_tok, cfg.H, cfg.dh), V.reshape(n_tok, cfg.H, cfg.dh), M,
+                        inp["scale"])
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def run_reference(args, ws, rank):
+    if rank != 0:
+        return
+    inp = W.make_layer(CFG)
+    n_tok = 1024
+    oracle_sample(inp, 256)  # import / first-touch
+    for _ in range(args.warmup):
+        oracle_sample(inp, n_tok)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample(inp, n_tok)
+    dt = (time.perf_counter() - t0) / args.steps
+    v = n_tok / dt
+    sample = (f"sequence 0 of the workload truncated to {n_tok} tokens, all {CFG.H} heads: float64 scan of K and V "
+              f"+ dense {n_tok}x{n_tok} M_test softmax attention")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(CFG, {"sample_tokens": n_tok}),
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def cpu_baseline():
+    inp = W.make_layer(CFG)
+    n_tok = 2048
+    oracle_sample(inp, 128)
+    t0 = time.perf_counter()
+    oracle_sample(inp, n_tok)
+    dt = time.perf_counter() - t0
+    return {"value": n_tok / dt, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"sequence 0 truncated to {n_tok} tokens, all {CFG.H} heads, one pass "
+                      f"(float64 scan of K and V + dense M_test attention), {dt:.1f} s"}
+
+
+# ------------------------------------------------------------------ CUDA path
+def run_ours(args, ws, rank, local):
+    from ssm_compressed_chunked_b200 import attamba as A, layer
+
+    dev = torch.device("cuda", local)
+    cfg = W.shrink(CFG, seed=CFG.seed + 1000 * rank) if ws > 1 else CFG
+    inp = W.make_layer(cfg)
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    nch = layer.n_chunks_of(cfg, inp["cu"])
+    pf = layer.Prefill(cfg.B, cfg.n, cfg.D, cfg.H, cfg.dh, cfg.N, nch, torch.bfloat16, dev)
+    mode = layer.mode_code(cfg.mode)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(events=None):
+        if events:
+            events[0].record(stream)
+        pf.index_step(None, cfg.P, cfg.offset, cfg.L, mode)
+        if events:
+            events[1].record(stream)
+        pf.scan_step(g["x"], g["dt_k"], g["dt_v"], g["bias_k"], g["bias_v"], g["A_k"], g["A_v"], g["B_k"],
+                     g["C_k"], g["B_v"], g["C_v"])
+        if events:
+            events[2].record(stream)
+        pf.attn_step(g["q"], inp["scale"])
+        if events:
+            events[3].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+
+    # algorithmic work of one step
+    T, D, N, H, dh = cfg.B * cfg.n, cfg.D, cfg.N, cfg.H, cfg.dh
+    ls = pf.index.ls.cpu().numpy().astype(np.int64)
+    nbb = pf.index.nbb.cpu().numpy().astype(np.int64)
+    i = np.tile(np.arange(cfg.n), cfg.B)
+    keys = int((nbb + np.maximum(0, i - ls + 1)).sum())
+    attn_flops = 4.0 * dh * H * keys
+    scan_bytes = T * (5 * D * 2 + 4 * N * 2) + 2 * nch * D * 2
+    scan_exps = 2.0 * T * D * N
+    index_bytes = T * 8 + nch * 8
+
+    sampler = ClockSampler(local) if rank == 0 else None
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)
+        step(evs[k])
+    torch.cuda.synchronize()
+    barrier(ws)
+    clocks = sampler.stop() if sampler else None
+
+    per = np.array([[evs[k][j].elapsed_time(evs[k][j + 1]) for j in range(3)] for k in range(args.steps)])  # ms
+    step_ms = per.sum(axis=1)
+    ms = max_over_ranks(float(step_ms.mean()), ws)
+    value = ws * T / (ms * 1e-3)
+
+    # end to end through the public API with host buffers: pinned H2D of the step's activations,
+    # the three calls, D2H of the output
+    names = ["x", "q", "dt_k", "dt_v", "B_k", "C_k", "B_v", "C_v"]
+    host = {k: inp[k].pin_memory() for k in names}
+    h_out = torch.empty(pf.O.shape, dtype=pf.O.dtype).pin_memory()
+    h2d = sum(host[k].numel() * host[k].element_size() for k in names)
+    d2h = h_out.numel() * h_out.element_size()
+    e2e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+
+    def e2e_step():
+        for k in names:
+            g[k].copy_(host[k], non_blocking=True)
+        step()
+        h_out.copy_(pf.O, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(3, min(args.steps, 10))
+    barrier(ws)
+    e2e_ev[0].record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e2e_ev[1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e2e_ev[0].elapsed_time(e2e_ev[1]) / e2e_steps, ws)
+    e2e_value = ws * T / (e2e_ms * 1e-3)
+
+    assert pf.status.item() == 0, f"device status {pf.status.item()}"
+    if rank != 0:
+        return
+
+    hbm, tf_burst, tf_sus, src = peaks()
+    mean = per.mean(axis=0)  # ms per launch: index, scan, attention
+    kernels = {
+        "chunk_index": {"ms": mean[0], "bytes": index_bytes},
+        "kv_ssm_scan": {"ms": mean[1], "bytes": scan_bytes, "exps": scan_exps},
+        "chunk_attn_fwd": {"ms": mean[2], "flops": attn_flops},
+    }
+    for k, d in kernels.items():
+        d["share"] = d["ms"] / mean.sum()
+    dom = max(kernels, key=lambda k: kernels[k]["ms"])
+    d = kernels[dom]
+    if dom == "chunk_attn_fwd":
+        ach = d["flops"] / (d["ms"] * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": tf_burst, "unit": "TFLOP/s", "frac": ach / tf_burst,
+                "peak_source": f"{src} bf16 burst"}
+        roof["traffic"] = ncu_traffic("chunk_attn_bf16_kernel")
+    else:
+        ach = d["bytes"] / (d["ms"] * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                "peak_source": f"{src} HBM copy"}
+        roof["traffic"] = ncu_traffic("kv_ssm_scan_kernel" if dom == "kv_ssm_scan" else "query_index_kernel")
+    roof["kernel"] = dom
+    # the scan's binding unit is the exponential: also report it against 16 ex2/clk/SM at the max SM clock
+    exp_peak = 16 * 148 * 1.965e9
+    scan = kernels["kv_ssm_scan"]
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) input, random-init projections)",
+        "config": config_block(cfg, {"parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"}),
+        "roofline": roof,
+        "kernels": {k: {"ms": round(v["ms"], 5), "share": round(v["share"], 4)} for k, v in kernels.items()},
+        "scan_exp_rate": {"achieved_Gexp_s": scan["exps"] / (scan["ms"] * 1e-3) / 1e9,
+                          "mufu_peak_Gexp_s": exp_peak / 1e9,
+                          "frac": scan["exps"] / (scan["ms"] * 1e-3) / exp_peak,
+                          "hbm_frac": scan["bytes"] / (scan["ms"] * 1e-3) / 1e9 / hbm},
+        "attn_tensor": {"achieved_TFLOP_s": attn_flops / (mean[2] * 1e-3) / 1e12,
+                        "frac_of_burst": attn_flops / (mean[2] * 1e-3) / 1e12 / tf_burst},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+    }
+    if ws == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        # the CPU oracle needs no process group: rank 0 times it, other ranks exit without work
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+        return
+    ws, rank, local = setup_dist()
+    try:
+        run_ours(args, ws, rank, local)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,77 @@
+"""Host-side checks of the C ABI (CPU only): the library loads, exports every
+declared symbol, and rejects bad arguments before touching the GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from ssm_compressed_chunked_b200 import attamba as A
+from ssm_compressed_chunked_b200 import workloads as W
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "attamba.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(attamba_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = A.load()
+    names = declared_functions()
+    assert set(names) == set(A.EXPORTS), names
+    for name in names:
+        assert hasattr(lib, name), name
+
+
+def test_version_and_status_strings():
+    assert "sm_100a" in A.version()
+    lib = A.load()
+    assert lib.attamba_status_string(0) == b"ok"
+    assert lib.attamba_status_string(1) == b"invalid argument"
+
+
+@pytest.mark.parametrize("n,P,o", [(10, 4, 0), (10, 4, 3), (256, 4, 0), (2048, 4, 3), (4096, 8, 0), (1, 4, 2),
+                                   (7, 1, 0), (9, 8, 7), (16, 16, 0)])
+def test_uniform_chunk_count_matches_workload_starts(n, P, o):
+    assert A.uniform_chunk_count(n, P, o) == len(W._uniform_starts(n, P, o))
+
+
+def test_invalid_arguments_are_rejected_on_the_host():
+    lib = A.load()
+    idx = A.IndexT(0, 0, 0, 0, 0, 4, 1, 16)
+    # no out arrays
+    assert lib.attamba_chunk_index(None, 4, 1, 16, 4, 0, 0, 0, ctypes.byref(idx), None, None) == A.ERR_INVALID_ARG
+    # wrong uniform chunk count
+    fake = 1 << 20
+    idx2 = A.IndexT(fake, fake, fake, fake, fake, 5, 1, 16)
+    assert lib.attamba_chunk_index(None, 5, 1, 16, 4, 0, 0, 0, ctypes.byref(idx2), None, None) == A.ERR_INVALID_ARG
+    # bad mode, negative L
+    idx3 = A.IndexT(fake, fake, fake, fake, fake, 4, 1, 16)
+    assert lib.attamba_chunk_index(None, 4, 1, 16, 4, 0, 0, 7, ctypes.byref(idx3), None, None) == A.ERR_INVALID_ARG
+    assert lib.attamba_chunk_index(None, 4, 1, 16, 4, 0, -1, 0, ctypes.byref(idx3), None, None) == A.ERR_INVALID_ARG
+    # scan: unsupported state size, misaligned pointer
+    p = [fake] * 12
+    assert lib.attamba_kv_ssm_scan(1, *p, 4, 16, 64, 32, fake, fake, None, None, None, None) == A.ERR_UNSUPPORTED
+    p_bad = [fake + 2] + [fake] * 11
+    assert lib.attamba_kv_ssm_scan(1, *p_bad, 4, 16, 64, 16, fake, fake, None, None, None, None) == A.ERR_INVALID_ARG
+    # attention: head_dim other than 64
+    assert lib.attamba_chunk_attn_fwd(1, fake, fake, fake, fake, fake, ctypes.byref(idx3), 2, 32,
+                                      ctypes.c_float(0.1), fake, None, None, None) == A.ERR_UNSUPPORTED
+    # decode: no leading tokens, f32 cache
+    c = A.CacheT(*([fake] * 8), 1, 1, 64, 16, 8, 0, 0, 16)
+    assert lib.attamba_decode_step(1, ctypes.byref(c), *([fake] * 12), ctypes.c_float(0.1), fake, fake,
+                                   1 << 20, None, None) == A.ERR_INVALID_ARG
+    c.L = 4
+    assert lib.attamba_decode_step(0, ctypes.byref(c), *([fake] * 12), ctypes.c_float(0.1), fake, fake,
+                                   1 << 20, None, None) == A.ERR_UNSUPPORTED
+    assert lib.attamba_decode_workspace_size(ctypes.byref(c)) > 0
+
+
+def test_cpu_tensors_are_refused():
+    import torch
+    with pytest.raises(A.AttambaError):
+        A._ptr(torch.zeros(4), None, "x")

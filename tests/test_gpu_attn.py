@@ -1,0 +1,96 @@
+"""GPU chunk-masked attention vs the oracle's dense masked softmax.
+
+Two levels: stage-isolated (the oracle attends over the GPU's own K/V, so the
+attention error is measured alone) and end to end (the oracle also runs the
+scan).  Cases span several 128-query tiles, ragged tails, tiny sequences, both
+masks, the empty-row case (M_test, L = 0), L >= n, P = 1 and variable chunks.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from helpers import assert_close, f64, oracle_attention_seq, oracle_scan_seq, run_prefill
+from ssm_compressed_chunked_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+C1, C2, C3 = W.LAYER_CONFIGS[1], W.LAYER_CONFIGS[2], W.LAYER_CONFIGS[3]
+SMALL = [
+    W.LAYER_CONFIGS[0],                                                    # fp32, full size
+    W.shrink(W.LAYER_CONFIGS[0], B=2, n=200, P=8, offset=3, L=5, mode="test"),   # fp32 M_test
+    W.shrink(C1, B=2, n=300, D=128, H=2),                                  # M_train, offset 3, L 4, ragged
+    W.shrink(C2, B=2, n=520, D=128, H=2),                                  # M_test P 8 L 64, 5 tiles
+    W.shrink(C3, B=2, n=387, D=128, H=2),                                  # variable chunks
+    W.shrink(C2, B=1, n=90, D=64, H=1),                                    # shorter than one tile
+    W.shrink(C2, B=2, n=260, D=64, H=1, L=0),                              # M_test, L = 0: empty rows
+    W.shrink(C1, B=1, n=200, D=64, H=1, L=500),                            # L >= n: causal
+    W.shrink(C1, B=1, n=256, D=128, H=2, P=1, offset=0, L=0),              # P = 1: causal
+    W.shrink(C2, B=2, n=384, D=128, H=2, P=64, L=3),                       # long chunks, M_test
+    W.shrink(C1, B=1, n=300, D=64, H=1, P=128, offset=17, L=0),            # long chunks, M_train
+]
+
+
+def _ids(c):
+    return f"{c.dtype}-{c.mode}-B{c.B}-n{c.n}-H{c.H}-P{c.P}-o{c.offset}-L{c.L}-{'var' if c.varlen else 'uni'}"
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=_ids)
+def test_attention_small(cfg):
+    inp = W.make_layer(cfg)
+    pf = run_prefill(inp, cfg)
+    n, H, dh = cfg.n, cfg.H, cfg.dh
+    O = pf.O.view(cfg.B, n, H, dh)
+    lse = pf.lse.cpu().numpy()
+    K = pf.K.view(cfg.B, n, H, dh)
+    V = pf.V.view(cfg.B, n, H, dh)
+    for b in range(cfg.B):
+        st = np.asarray(inp["starts"][b])
+        q = f64(inp["q"][b])
+        # stage-isolated: oracle attention over the GPU's own K/V
+        ro, rl = oracle_attention_seq(q, f64(K[b]), f64(V[b]), st, n, cfg.L, cfg.mode, inp["scale"])
+        assert_close(cfg.dtype, f64(O[b]), ro, f"O (isolated) b={b}")
+        fin = np.isfinite(rl)
+        assert np.array_equal(np.isfinite(lse[b]), fin)
+        assert_close(cfg.dtype, lse[b][fin], rl[fin], f"lse b={b}")
+        # end to end: oracle scan + oracle attention
+        rk, rv = oracle_scan_seq(inp, b)
+        eo, _ = oracle_attention_seq(q, rk.reshape(n, H, dh), rv.reshape(n, H, dh), st, n, cfg.L, cfg.mode,
+                                     inp["scale"])
+        assert_close(cfg.dtype, f64(O[b]), eo, f"O (end to end) b={b}")
+    assert pf.status.item() == 0
+
+
+@pytest.mark.parametrize("cfg", [C1, C2, C3], ids=lambda c: c.name)
+def test_attention_full_size_sampled_rows(cfg):
+    """Full-size configs in the bench's launch configuration; the oracle recomputes sampled query rows."""
+    inp = W.make_layer(cfg)
+    pf = run_prefill(inp, cfg)
+    n, H, dh = cfg.n, cfg.H, cfg.dh
+    O = pf.O.view(cfg.B, n, H, dh)
+    K = pf.K.view(cfg.B, n, H, dh)
+    V = pf.V.view(cfg.B, n, H, dh)
+    rng = np.random.default_rng(7)
+    b = cfg.B - 1
+    st = np.asarray(inp["starts"][b])
+    rows = sorted({0, 1, 127, 128, n - 129, n - 1} | set(rng.integers(0, n, size=26).tolist()))
+    q = f64(inp["q"][b])
+    ro, _ = oracle_attention_seq(q, f64(K[b]), f64(V[b]), st, n, cfg.L, cfg.mode, inp["scale"], rows)
+    assert_close(cfg.dtype, f64(O[b])[rows], ro, "O (isolated, sampled)")
+    rk, rv = oracle_scan_seq(inp, b)
+    eo, _ = oracle_attention_seq(q, rk.reshape(n, H, dh), rv.reshape(n, H, dh), st, n, cfg.L, cfg.mode,
+                                 inp["scale"], rows)
+    assert_close(cfg.dtype, f64(O[b])[rows], eo, "O (end to end, sampled)")
+    assert pf.status.item() == 0
+
+
+def test_value_one_gives_output_one():
+    """V == 1 everywhere gives O == 1 on every row with a key (softmax weights sum to one)."""
+    cfg = W.shrink(C2, B=2, n=300, D=128, H=2)
+    inp = W.make_layer(cfg)
+    pf = run_prefill(inp, cfg)
+    pf.V.fill_(1.0)
+    pf.Vc.fill_(1.0)
+    pf.attn_step(inp["q"].cuda(), inp["scale"])
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(f64(pf.O), 1.0, atol=1e-2)

@@ -1,0 +1,58 @@
+"""GPU KV-SSM scan vs the oracle's per-token recurrence."""
+
+import numpy as np
+import pytest
+import torch
+
+from helpers import assert_close, f64, oracle_scan_seq, run_prefill
+from oracle import chunks as OC
+from ssm_compressed_chunked_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    W.LAYER_CONFIGS[0],                                                   # fp32, full size
+    W.shrink(W.LAYER_CONFIGS[1], B=2, n=300, D=128, H=2),                 # cyclic offset 3, ragged n
+    W.shrink(W.LAYER_CONFIGS[2], B=2, n=333, D=192, H=3),                 # P = 8
+    W.shrink(W.LAYER_CONFIGS[3], B=3, n=257, D=128, H=2),                 # variable chunks
+    W.shrink(W.LAYER_CONFIGS[1], B=1, n=64, D=64, H=1, P=1, offset=0),   # P = 1
+    W.shrink(W.LAYER_CONFIGS[1], B=2, n=50, D=64, H=1, P=64, offset=0),  # one chunk per sequence
+    W.shrink(W.LAYER_CONFIGS[0], B=2, n=77, D=64, H=1, P=16, offset=5),   # fp32 cyclic
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: f"{c.name}-B{c.B}-n{c.n}-D{c.D}-P{c.P}")
+def test_scan_small(cfg):
+    inp = W.make_layer(cfg)
+    pf = run_prefill(inp, cfg)
+    K = pf.K.view(cfg.B, cfg.n, cfg.D)
+    V = pf.V.view(cfg.B, cfg.n, cfg.D)
+    for b in range(cfg.B):
+        rk, rv = oracle_scan_seq(inp, b)
+        assert_close(cfg.dtype, f64(K[b]), rk, f"K b={b}")
+        assert_close(cfg.dtype, f64(V[b]), rv, f"V b={b}")
+    # chunk-end rows are the same values as the full outputs at the chunk ends (bit-exact copy)
+    ends = np.array([b * cfg.n + e for b, st in enumerate(inp["starts"]) for e in OC.boundary_positions(st, cfg.n)])
+    assert torch.equal(pf.Kc, pf.K[torch.from_numpy(ends).cuda()])
+    assert torch.equal(pf.Vc, pf.V[torch.from_numpy(ends).cuda()])
+    assert pf.status.item() == 0
+
+
+@pytest.mark.parametrize("ci", [1, 2, 3])
+def test_scan_full_size_sampled_chunks(ci):
+    """Configs at full size, in the launch the bench times; the oracle recomputes sampled chunks."""
+    cfg = W.LAYER_CONFIGS[ci]
+    inp = W.make_layer(cfg)
+    pf = run_prefill(inp, cfg)
+    K = pf.K.view(cfg.B, cfg.n, cfg.D)
+    V = pf.V.view(cfg.B, cfg.n, cfg.D)
+    rng = np.random.default_rng(ci)
+    for b in (0, cfg.B - 1):
+        st = list(inp["starts"][b]) + [cfg.n]
+        picks = {0, len(st) - 2} | set(rng.integers(0, len(st) - 1, size=4).tolist())
+        for c in sorted(picks):
+            t0, t1 = st[c], st[c + 1]
+            rk, rv = oracle_scan_seq(inp, b, t0, t1)
+            assert_close(cfg.dtype, f64(K[b, t0:t1]), rk, f"K b={b} chunk={c}")
+            assert_close(cfg.dtype, f64(V[b, t0:t1]), rv, f"V b={b} chunk={c}")
+    assert pf.status.item() == 0
