@@ -54,50 +54,61 @@ def config_block(cfg, extra=None):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+    """SM clock and clock-event (throttle) reasons sampled through NVML every ~2 ms in a thread.
+
+    mark() opens the window whose samples are reported (the timed region)."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
     def __init__(self, gpu_index):
-        self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        import threading
+        self.samples, self.t_mark = [], None
+        self.stop_evt = threading.Event()
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=self.f, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            try:  # NVML indexes physical devices: find ours by PCI address
+                pr = torch.cuda.get_device_properties(gpu_index)
+                bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: no clock record
+            self.nv = None
+            return
+        self.th = threading.Thread(target=self._run, daemon=True)
+        self.th.start()
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_evt.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def mark(self):
+        self.t_mark = time.perf_counter()
 
     def stop(self):
-        if self.proc is None:
+        if self.nv is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.f.close()
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
+        self.stop_evt.set()
+        self.th.join(timeout=2)
+        win = [x for x in self.samples if self.t_mark is None or x[0] >= self.t_mark]
+        if len(win) < 3:  # a very short timed region: widen to the last 0.5 s before it
+            win = [x for x in self.samples if self.t_mark is None or x[0] >= self.t_mark - 0.5]
+        if not win:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = sorted(k for k, bit in self.REASONS.items() if any(r & bit for _, _, r in win))
+        return {"sm_mhz": statistics.median(m for _, m, _ in win), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(win), "source": "NVML, 2 ms period"}
 
 
 def source_sha(files):
@@ -141,6 +152,16 @@ def max_over_ranks(x, ws):
     t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_config(cfg, ws, rank):
+    """Each rank runs its own batch of the workload (weak scaling): same shapes, its own seed."""
+    return W.shrink(cfg, seed=cfg.seed + 1000 * rank) if ws > 1 else cfg
+
+
+def job_throughput(ws, tokens_per_rank, max_ms):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return ws * tokens_per_rank / (max_ms * 1e-3)
 
 
 def barrier(ws):
@@ -216,7 +237,7 @@ def run_ours(args, ws, rank, local):
     from ssm_compressed_chunked_b200 import attamba as A, layer
 
     dev = torch.device("cuda", local)
-    cfg = W.shrink(CFG, seed=CFG.seed + 1000 * rank) if ws > 1 else CFG
+    cfg = rank_config(CFG, ws, rank)
     inp = W.make_layer(cfg)
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
     nch = layer.n_chunks_of(cfg, inp["cu"])
@@ -239,9 +260,15 @@ def run_ours(args, ws, rank, local):
         if events:
             events[3].record(stream)
 
-    for _ in range(max(3, args.warmup)):
+    sampler = ClockSampler(local) if rank == 0 else None
+    t_w = time.perf_counter()
+    nw = 0
+    while nw < max(3, args.warmup) or (time.perf_counter() - t_w) * 1e3 < args.min_warmup_ms:
         flush.fill_(1)
         step()
+        nw += 1
+        if nw % 16 == 0:
+            torch.cuda.synchronize()
     torch.cuda.synchronize()
 
     # algorithmic work of one step
@@ -255,10 +282,11 @@ def run_ours(args, ws, rank, local):
     scan_exps = 2.0 * T * D * N
     index_bytes = T * 8 + nch * 8
 
-    sampler = ClockSampler(local) if rank == 0 else None
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     barrier(ws)
     torch.cuda.synchronize()
+    if sampler:
+        sampler.mark()
     for k in range(args.steps):
         flush.fill_(k & 0xFF)
         step(evs[k])
@@ -269,7 +297,7 @@ def run_ours(args, ws, rank, local):
     per = np.array([[evs[k][j].elapsed_time(evs[k][j + 1]) for j in range(3)] for k in range(args.steps)])  # ms
     step_ms = per.sum(axis=1)
     ms = max_over_ranks(float(step_ms.mean()), ws)
-    value = ws * T / (ms * 1e-3)
+    value = job_throughput(ws, T, ms)
 
     # end to end through the public API with host buffers: pinned H2D of the step's activations,
     # the three calls, D2H of the output
@@ -297,7 +325,7 @@ def run_ours(args, ws, rank, local):
     e2e_ev[1].record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e2e_ev[0].elapsed_time(e2e_ev[1]) / e2e_steps, ws)
-    e2e_value = ws * T / (e2e_ms * 1e-3)
+    e2e_value = job_throughput(ws, T, e2e_ms)
 
     assert pf.status.item() == 0, f"device status {pf.status.item()}"
     if rank != 0:
@@ -357,6 +385,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--min-warmup-ms", type=float, default=500.0,
+                    help="keep warming up at least this long so clocks have ramped (0 under a profiler)")
     args = ap.parse_args()
     if args.impl == "reference":
         # the CPU oracle needs no process group: rank 0 times it, other ranks exit without work

@@ -8,16 +8,28 @@
 // ends (nbb(i) of them, stored contiguously in Kc/Vc) and a contiguous local
 // segment [ls(i), i] of the full K/V.
 //
-// bf16 kernel (tcgen05): one CTA per (128 queries, head, sequence).  Its key
-// tiles (128 keys each) are first the chunk-end tiles 0..nbb(last query), then
+// bf16 kernel (tcgen05), persistent: two CTAs per SM walk work items of 128
+// queries of one (sequence, head), longest key lists first.  An item's key
+// tiles (64 keys each) are first the chunk-end tiles 0..nbb(last query), then
 // the local band [ls(first query), last query]; both are plain TMA boxes.
-//   warp 4     TMA producer: Q once, then K/V tiles into a 2-stage ring
-//   warp 5     one thread issues tcgen05.mma: S = Q K^T (M128 N128 K64) into
-//              TMEM, then O_j = P_j V_j (M128 N64 K128) into TMEM
-//   warps 0-3  softmax, one query row per thread: tcgen05.ld of its S row,
-//              mask, online max/sum in fp32, P as bf16 into shared memory
-//              (the A operand of the PV MMA), then accumulate O_j in registers
-// TMEM: S double buffer (2 x 128 columns) + O_j double buffer (2 x 64).
+//   warp 4     TMA producer: Q (double buffered across items), then K/V tiles
+//              into a 3-stage ring
+//   warp 5     one thread issues tcgen05.mma: S = Q K^T (M128 N64 K64) into
+//              TMEM, then O += P_j V_j (M128 N64 K64) into TMEM
+//   warps 0-3  softmax, one query row per thread: one tcgen05.ld round trip for
+//              its S row, masking only where a row's key range cuts the tile,
+//              32-column chunks outside every row's range skipped, online
+//              max/sum in fp32, P as bf16 into shared memory (the A operand of
+//              the PV MMA)
+// O accumulates in TMEM across an item's tiles.  P uses a reference max that
+// is raised (and O, l rescaled in TMEM) only when a row's max grows by more
+// than 2^8, so P <= 2^8 and the rescale is rare; the final O / l is exact
+// whatever reference was used.  Tile counters run across items, so the next
+// item's loads and QK^T overlap the current item's softmax and epilogue.
+// TMEM per CTA: S double buffer (2 x 64 columns) + O accumulators (2 x 64, by
+// item parity) = 256 columns, so two CTAs share an SM's 512; shared memory per
+// CTA: Q x 2, K/V x 3 stages, one P buffer (the next tile's softmax reaches its
+// P write only after the previous PV has finished).
 // Every wait is bounded; on a give-up the CTA raises ATTAMBA_DEV_TIMEOUT,
 // drains its own copies and MMAs, frees TMEM and leaves the tile unwritten.
 //
@@ -32,87 +44,161 @@
 namespace attamba {
 
 namespace {
-constexpr int kBM = 128;
-constexpr int kBN = 128;
+constexpr int kBM = 128;                                    // queries per work item (TMEM lanes)
+constexpr int kBN = 64;                                     // keys per tile
 constexpr int kDH = 64;
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kThreads = 192;
-constexpr uint32_t kTileBytes = kBN * kDH * 2;    // 16 KB: 128 rows x 128 bytes
-constexpr uint32_t kQOff = 0;
-constexpr uint32_t kKOff = kQOff + kTileBytes;              // 2 stages
-constexpr uint32_t kVOff = kKOff + kStages * kTileBytes;    // 2 stages
-constexpr uint32_t kPOff = kVOff + kStages * kTileBytes;    // 2 buffers x 2 column blocks
-constexpr uint32_t kPBytes = 2 * kTileBytes;                // 128 rows x 128 keys bf16
-constexpr uint32_t kBarOff = kPOff + 2 * kPBytes;
-constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;       // + barriers + alignment slack
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSCol = 0;     // S buffers at columns 0 and 128
-constexpr uint32_t kOCol = 256;   // O buffers at columns 256 and 320
+constexpr int kCtasPerSm = 2;
+constexpr int kMaxItems = 64;                               // work items per CTA (the host sizes the grid)
+constexpr uint32_t kQBytes = kBM * kDH * 2;                 // 16 KB: 128 rows x 128 bytes
+constexpr uint32_t kKVBytes = kBN * kDH * 2;                // 8 KB: 64 rows x 128 bytes
+constexpr uint32_t kPBytes = kBM * kBN * 2;                 // 16 KB: 128 rows x 64 keys bf16
+constexpr uint32_t kQOff = 0;                               // 2 Q buffers
+constexpr uint32_t kKOff = kQOff + 2 * kQBytes;             // kStages K tiles
+constexpr uint32_t kVOff = kKOff + kStages * kKVBytes;      // kStages V tiles
+constexpr uint32_t kPOff = kVOff + kStages * kKVBytes;      // 1 P buffer
+constexpr uint32_t kBarOff = kPOff + kPBytes;
+constexpr uint32_t kItemOff = kBarOff + 256;
+constexpr uint32_t kSmemBytes = kItemOff + kMaxItems * 32 + 1024;   // + item table + alignment slack
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kSCol = 0;     // S buffers at columns 0 and 64
+constexpr uint32_t kOCol = 128;   // O accumulators at columns 128 and 192 (by item parity)
 constexpr uint64_t kWaitNs = 4000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescale = 8.f;   // O is rescaled only when a row's max grows by more than 2^8
 
 struct Bars {
-  uint64_t q_full;
+  uint64_t q_full[2];
+  uint64_t q_empty[2];
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
   uint64_t s_full[2];
   uint64_t p_full[2];
-  uint64_t o_full[2];
-  uint64_t o_empty[2];
+  uint64_t pv_done[2];   // PV of global tile g completes phase g/2 of pv_done[g & 1]
+  uint64_t o_empty[2];   // the epilogue has read O accumulator [item parity]
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+// One work item: 128 queries of one (sequence, head).  Items are numbered so
+// that the longest key lists (last query tiles) come first.
+struct Item {
+  int b, h, q0, q_last, ls_first, nbt, NT, chunk0;
+};
+
+__device__ __forceinline__ Item decode_item(const AttnArgs& a, int item, int n_qt) {
+  const int BH = a.B * a.H;
+  const int qt = n_qt - 1 - item / BH;
+  const int bh = item - (item / BH) * BH;
+  Item it;
+  it.b = bh / a.H;
+  it.h = bh - it.b * a.H;
+  it.q0 = qt * kBM;
+  it.q_last = min(it.q0 + kBM, a.n) - 1;
+  const int64_t tok0 = (int64_t)it.b * a.n;
+  it.ls_first = a.ls[tok0 + it.q0];
+  it.nbt = (a.nbb[tok0 + it.q_last] + kBN - 1) / kBN;
+  // the local segment [ls(i), i] is empty only when ls(i) = i + 1 (M_test, L = 0);
+  // ls(i) - i does not grow with i, so the last row decides
+  const bool band_empty = a.ls[tok0 + it.q_last] > it.q_last;
+  const int band_len = band_empty ? 0 : max(0, it.q_last - it.ls_first + 1);
+  it.NT = it.nbt + (band_len + kBN - 1) / kBN;
+  it.chunk0 = a.bptr[it.b];
+  return it;
+}
+
+// 128 consecutive 32-bit TMEM columns of this thread's lane, one wait
+__device__ __forceinline__ void tmem_ld128_sync(uint32_t taddr, uint32_t (&r)[128]) {
+#define ATT_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), "=r"(r[i + 5]), \
+                  "=r"(r[i + 6]), "=r"(r[i + 7])
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%128];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,"
+      "%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%129];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,"
+      "%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95}, [%130];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,"
+      "%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, "
+      "[%131];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : ATT_R8(0), ATT_R8(8), ATT_R8(16), ATT_R8(24), ATT_R8(32), ATT_R8(40), ATT_R8(48), ATT_R8(56),
+        ATT_R8(64), ATT_R8(72), ATT_R8(80), ATT_R8(88), ATT_R8(96), ATT_R8(104), ATT_R8(112), ATT_R8(120)
+      : "r"(taddr), "r"(taddr + 32), "r"(taddr + 64), "r"(taddr + 96)
+      : "memory");
+#undef ATT_R8
+}
+
+// 32 consecutive 32-bit columns from registers into this thread's TMEM lane, waited
+__device__ __forceinline__ void tmem_st32_sync(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(reinterpret_cast<uint64_t&>(d))
+      : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)),
+        "l"(reinterpret_cast<const uint64_t&>(c)));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("add.rn.f32x2 %0, %1, %2;"
+      : "=l"(reinterpret_cast<uint64_t&>(d))
+      : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)));
+  return d;
+}
+
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     chunk_attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc,
                            const __grid_constant__ CUtensorMap tm_vc, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);
+  Item* items = reinterpret_cast<Item*>(smem + kItemOff);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qt = gridDim.x - 1 - blockIdx.x;  // longest key lists first
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int n = a.n, H = a.H;
-  const int q0 = qt * kBM;
-  const int q_last = min(q0 + kBM, n) - 1;
-  const int64_t tok0 = (int64_t)b * n;
-
-  const int ls_first = a.ls[tok0 + q0];
-  const int nbb_last = a.nbb[tok0 + q_last];
-  const int nbt = (nbb_last + kBN - 1) / kBN;
-  // every row's local segment [ls(i), i] is empty only when ls(i) = i + 1 (M_test, L = 0);
-  // ls(i) - i does not grow with i, so the last row decides
-  const bool band_empty = a.ls[tok0 + q_last] > q_last;
-  const int band_len = band_empty ? 0 : max(0, q_last - ls_first + 1);
-  const int nband = (band_len + kBN - 1) / kBN;
-  const int NT = nbt + nband;
-  const int32_t chunk0 = a.bptr[b];
-
+  const int n_qt = (a.n + kBM - 1) / kBM;
+  const int n_items_all = n_qt * a.B * a.H;
+  // this CTA's items: blockIdx.x, blockIdx.x + gridDim.x, ...
+  const int my_items = (n_items_all - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+  const int H = a.H, n = a.n;
   __nv_bfloat16* O = static_cast<__nv_bfloat16*>(a.O);
-  if (NT == 0) {  // every row of the tile has an empty key set
-    if (tid < kBM && q0 + tid <= q_last) {
-      const int i = q0 + tid;
-      uint4* dst = reinterpret_cast<uint4*>(O + ((tok0 + i) * H + h) * kDH);
-#pragma unroll
-      for (int c = 0; c < kDH / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
-      if (a.lse) a.lse[((int64_t)b * H + h) * n + i] = -INFINITY;
-    }
+
+  if (my_items > kMaxItems) {  // the host sizes the grid so that this cannot happen
+    if (tid == 0) raise_status(a.status, ATTAMBA_DEV_TIMEOUT);
     return;
   }
-
+  for (int k = tid; k < my_items; k += kThreads) items[k] = decode_item(a, blockIdx.x + k * gridDim.x, n_qt);
   if (warp == 4 && lane == 0) {
-    mbar_init(&bars->q_full, 1);
-    for (int i = 0; i < kStages; ++i) { mbar_init(&bars->kv_full[i], 1); mbar_init(&bars->kv_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->q_full[i], 1);
+      mbar_init(&bars->q_empty[i], 1);
       mbar_init(&bars->s_full[i], 1);
       mbar_init(&bars->p_full[i], kBM);
-      mbar_init(&bars->o_full[i], 1);
+      mbar_init(&bars->pv_done[i], 1);
       mbar_init(&bars->o_empty[i], kBM);
     }
+    for (int i = 0; i < kStages; ++i) { mbar_init(&bars->kv_full[i], 1); mbar_init(&bars->kv_empty[i], 1); }
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -132,31 +218,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_kc); tma_prefetch_desc(&tm_vc);
-      mbar_arrive_expect_tx(&bars->q_full, kTileBytes);
-      tma_load_3d(smem + kQOff, &tm_q, 0, h, (int)(tok0 + q0), &bars->q_full);
-      int issued = 0;
-      for (int j = 0; j < NT; ++j) {
-        const int st = j % kStages;
-        if (j >= kStages &&
-            !mbar_wait_bounded(&bars->kv_empty[st], ((j / kStages) - 1) & 1, abort_flag, kWaitNs)) {
-          *abort_flag = 1;
+      int g = 0, wi = 0;
+      bool ok = true;
+      for (int k = 0; ok && k < my_items; ++k) {
+        const Item it = items[k];
+        if (it.NT == 0) continue;
+        const int64_t tok0 = (int64_t)it.b * n;
+        const int qb = wi & 1;
+        if (wi >= 2 && !mbar_wait_bounded(&bars->q_empty[qb], ((wi - 2) >> 1) & 1, abort_flag, kWaitNs)) {
+          ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&bars->kv_full[st], 2 * kTileBytes);
-        if (j < nbt) {
-          const int row = chunk0 + j * kBN;
-          tma_load_3d(smem + kKOff + st * kTileBytes, &tm_kc, 0, h, row, &bars->kv_full[st]);
-          tma_load_3d(smem + kVOff + st * kTileBytes, &tm_vc, 0, h, row, &bars->kv_full[st]);
-        } else {
-          const int row = (int)(tok0 + ls_first + (j - nbt) * kBN);
-          tma_load_3d(smem + kKOff + st * kTileBytes, &tm_k, 0, h, row, &bars->kv_full[st]);
-          tma_load_3d(smem + kVOff + st * kTileBytes, &tm_v, 0, h, row, &bars->kv_full[st]);
+        mbar_arrive_expect_tx(&bars->q_full[qb], kQBytes);
+        tma_load_3d(smem + kQOff + qb * kQBytes, &tm_q, 0, it.h, (int)(tok0 + it.q0), &bars->q_full[qb]);
+        ++wi;
+        for (int j = 0; j < it.NT; ++j, ++g) {
+          const int st = g % kStages;
+          if (g >= kStages &&
+              !mbar_wait_bounded(&bars->kv_empty[st], ((g / kStages) - 1) & 1, abort_flag, kWaitNs)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bars->kv_full[st], 2 * kKVBytes);
+          if (j < it.nbt) {
+            const int row = it.chunk0 + j * kBN;
+            tma_load_3d(smem + kKOff + st * kKVBytes, &tm_kc, 0, it.h, row, &bars->kv_full[st]);
+            tma_load_3d(smem + kVOff + st * kKVBytes, &tm_vc, 0, it.h, row, &bars->kv_full[st]);
+          } else {
+            const int row = (int)(tok0 + it.ls_first + (j - it.nbt) * kBN);
+            tma_load_3d(smem + kKOff + st * kKVBytes, &tm_k, 0, it.h, row, &bars->kv_full[st]);
+            tma_load_3d(smem + kVOff + st * kKVBytes, &tm_v, 0, it.h, row, &bars->kv_full[st]);
+          }
         }
-        issued = j + 1;
       }
-      // drain: the last loads of each stage must land before the CTA may exit
-      mbar_wait_timeout(&bars->q_full, 0, kWaitNs);
-      for (int j = max(0, issued - kStages); j < issued; ++j)
+      if (!ok) *abort_flag = 1;
+      // drain: the last copies into each buffer must land before the CTA may exit
+      for (int w = max(0, wi - 2); w < wi; ++w) mbar_wait_timeout(&bars->q_full[w & 1], (w >> 1) & 1, kWaitNs);
+      for (int j = max(0, g - kStages); j < g; ++j)
         mbar_wait_timeout(&bars->kv_full[j % kStages], (j / kStages) & 1, kWaitNs);
     }
   } else if (warp == 5) {
@@ -164,43 +262,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_qk = umma_idesc_bf16(kBM, kBN, 0, 0);
       const uint32_t idesc_pv = umma_idesc_bf16(kBM, kDH, 0, 1);
-      const uint32_t sq = smem_u32(smem + kQOff);
-      bool ok = mbar_wait_bounded(&bars->q_full, 0, abort_flag, kWaitNs);
-      auto issue_pv = [&](int jj) -> bool {
-        const int sb = jj & 1, st = jj % kStages;
-        if (!mbar_wait_bounded(&bars->p_full[sb], (jj >> 1) & 1, abort_flag, kWaitNs)) return false;
-        if (jj >= 2 && !mbar_wait_bounded(&bars->o_empty[sb], ((jj - 2) >> 1) & 1, abort_flag, kWaitNs))
+      // PV of tile gg into the O accumulator of item wi_of (first tile of the item overwrites)
+      auto issue_pv = [&](int gg, int wi_of, bool first) -> bool {
+        const int sb = gg & 1, st = gg % kStages, ob = wi_of & 1;
+        if (!mbar_wait_bounded(&bars->p_full[sb], (gg >> 1) & 1, abort_flag, kWaitNs)) return false;
+        if (first && wi_of >= 2 &&
+            !mbar_wait_bounded(&bars->o_empty[ob], ((wi_of - 2) >> 1) & 1, abort_flag, kWaitNs))
           return false;
         tc_fence_after();
-        const uint32_t sp = smem_u32(smem + kPOff + sb * kPBytes);
-        const uint32_t sv = smem_u32(smem + kVOff + st * kTileBytes);
+        const uint32_t sp = smem_u32(smem + kPOff);
+        const uint32_t sv = smem_u32(smem + kVOff + st * kKVBytes);
 #pragma unroll
         for (int k = 0; k < kBN / 16; ++k) {
-          // A = P (K-major: 64-key column blocks of 16 KB, 32 bytes per 16 keys)
-          const uint64_t adesc = umma_desc_sw128(sp + (k >> 2) * kTileBytes + (k & 3) * 32, 16, 1024);
+          // A = P (K-major: 128 rows x 64 keys, 32 bytes per 16 keys)
+          const uint64_t adesc = umma_desc_sw128(sp + k * 32, 16, 1024);
           // B = V (MN-major: 16 keys = two 8-row groups of 1024 bytes)
           const uint64_t bdesc = umma_desc_sw128(sv + k * 2048, 16, 1024);
-          umma_bf16(tmem + kOCol + sb * kDH, adesc, bdesc, idesc_pv, k > 0 ? 1u : 0u);
+          umma_bf16(tmem + kOCol + ob * kDH, adesc, bdesc, idesc_pv, (first && k == 0) ? 0u : 1u);
         }
-        umma_commit(&bars->o_full[sb]);
+        umma_commit(&bars->pv_done[sb]);
         umma_commit(&bars->kv_empty[st]);
         return true;
       };
-      for (int j = 0; ok && j < NT; ++j) {
-        const int st = j % kStages, sb = j & 1;
-        if (!mbar_wait_bounded(&bars->kv_full[st], (j / kStages) & 1, abort_flag, kWaitNs)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t sk = smem_u32(smem + kKOff + st * kTileBytes);
+      int g = 0, wi = 0;
+      int pend_wi = 0;
+      bool pend_first = false;
+      bool ok = true;
+      for (int k = 0; ok && k < my_items; ++k) {
+        const Item it = items[k];
+        if (it.NT == 0) continue;
+        const int qb = wi & 1;
+        if (!mbar_wait_bounded(&bars->q_full[qb], (wi >> 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
+        const uint32_t sq = smem_u32(smem + kQOff + qb * kQBytes);
+        for (int j = 0; j < it.NT; ++j, ++g) {
+          const int st = g % kStages, sb = g & 1;
+          if (!mbar_wait_bounded(&bars->kv_full[st], (g / kStages) & 1, abort_flag, kWaitNs)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sk = smem_u32(smem + kKOff + st * kKVBytes);
 #pragma unroll
-        for (int k = 0; k < kDH / 16; ++k) {
-          const uint64_t adesc = umma_desc_sw128(sq + k * 32, 16, 1024);
-          const uint64_t bdesc = umma_desc_sw128(sk + k * 32, 16, 1024);
-          umma_bf16(tmem + kSCol + sb * kBN, adesc, bdesc, idesc_qk, k > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kDH / 16; ++kk) {
+            const uint64_t adesc = umma_desc_sw128(sq + kk * 32, 16, 1024);
+            const uint64_t bdesc = umma_desc_sw128(sk + kk * 32, 16, 1024);
+            umma_bf16(tmem + kSCol + sb * kBN, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&bars->s_full[sb]);
+          if (j == it.NT - 1) umma_commit(&bars->q_empty[qb]);  // Q buffer free once its last QK is done
+          if (g >= 1 && !issue_pv(g - 1, pend_wi, pend_first)) { ok = false; break; }
+          pend_wi = wi;
+          pend_first = (j == 0);
         }
-        umma_commit(&bars->s_full[sb]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        ++wi;
       }
-      if (ok) ok = issue_pv(NT - 1);
+      if (ok && g >= 1) ok = issue_pv(g - 1, pend_wi, pend_first);
       if (!ok) *abort_flag = 1;
       umma_commit(&bars->mma_done);  // every MMA issued above has finished when this arrives
       mbar_wait_timeout(&bars->mma_done, 0, kWaitNs);
@@ -208,119 +321,182 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax warps 0-3
     const int r = tid;  // query row within the tile == TMEM lane
-    const int i = q0 + r;
-    const bool row_ok = i <= q_last;
-    const int my_ls = row_ok ? a.ls[tok0 + i] : 0;
-    const int my_nbb = row_ok ? a.nbb[tok0 + i] : 0;
     const float sl2 = a.scale * kLog2e;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    uint8_t* p_row_base = smem + kPOff + r * 128;
+    uint8_t* prow = smem + kPOff + r * 128;
     const int sw = r & 7;
-
-    float m_run = -INFINITY, l_run = 0.f;
-    float m_acc_use = 0.f;
-    bool acc_empty = true;
-    float acc[kDH];
-#pragma unroll
-    for (int c = 0; c < kDH; ++c) acc[c] = 0.f;
-    float m_tile_use = 0.f;  // running-max reference used for the previous tile's P
+    int g = 0, wi = 0;
     bool ok = true;
-
-    auto accumulate = [&](int jj, float m_ref) -> bool {
-      const int ob = jj & 1;
-      if (!mbar_wait_bounded(&bars->o_full[ob], (jj >> 1) & 1, abort_flag, kWaitNs)) return false;
+    // wait for the PV of global tile gg (consecutive waits per P buffer; verdict warp-uniform)
+    auto wait_pv = [&](int gg) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done[gg & 1], (gg >> 1) & 1, abort_flag, kWaitNs));
+    };
+    // this row's key range of the first item, then prefetched one item ahead
+    int nx_ls = 0, nx_nbb = 0;
+    if (my_items > 0 && items[0].q0 + r <= items[0].q_last) {
+      const int64_t tok = (int64_t)items[0].b * n + items[0].q0 + r;
+      nx_ls = a.ls[tok];
+      nx_nbb = a.nbb[tok];
+    }
+    for (int k = 0; ok && k < my_items; ++k) {
+      const Item it = items[k];
+      const int64_t tok0 = (int64_t)it.b * n;
+      const int i = it.q0 + r;
+      const bool row_ok = i <= it.q_last;
+      const int my_ls = nx_ls, my_nbb = nx_nbb;
+      if (k + 1 < my_items) {
+        const Item nx = items[k + 1];
+        if (nx.q0 + r <= nx.q_last) {
+          const int64_t tok = (int64_t)nx.b * n + nx.q0 + r;
+          nx_ls = a.ls[tok];
+          nx_nbb = a.nbb[tok];
+        }
+      }
+      if (it.NT == 0) {  // every row of the item has an empty key set
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(O + ((tok0 + i) * H + it.h) * kDH);
+#pragma unroll
+          for (int c = 0; c < kDH / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+          if (a.lse) a.lse[((int64_t)it.b * H + it.h) * n + i] = -INFINITY;
+        }
+        continue;
+      }
+      const int ob = wi & 1;
+      const uint32_t o_tmem = lane_base + kOCol + ob * kDH;
+      float m_ref = -INFINITY, l_run = 0.f;  // P of this item is exp2(s * sl2 - m_ref)
+      for (int j = 0; j < it.NT; ++j, ++g) {
+        const int sb = g & 1;
+        int lo, hi;
+        if (j < it.nbt) {
+          lo = 0;
+          hi = min(max(my_nbb - j * kBN, 0), kBN);
+        } else {
+          const int j0 = it.ls_first + (j - it.nbt) * kBN;
+          lo = min(max(my_ls - j0, 0), kBN);
+          hi = min(max(i - j0 + 1, 0), kBN);
+        }
+        if (!row_ok) { lo = 0; hi = 0; }
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[sb], (g >> 1) & 1, abort_flag, kWaitNs))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sr[kBN];
+        tmem_ld32_sync(lane_base + kSCol + sb * kBN, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32_sync(lane_base + kSCol + sb * kBN + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        float s[kBN];
+        // row max of the raw scores over the valid columns [lo, hi)
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+        if (lo == 0 && hi == kBN) {
+#pragma unroll
+          for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c]);
+        } else {
+          const unsigned span = (unsigned)(hi - lo);
+#pragma unroll
+          for (int c = 0; c < kBN; ++c)
+            s[c] = ((unsigned)(c - lo) < span) ? __uint_as_float(sr[c]) : -INFINITY;
+        }
+#pragma unroll
+        for (int c = 0; c < kBN; c += 8) {
+          mx0 = max3(mx0, s[c], s[c + 1]);
+          mx1 = max3(mx1, s[c + 2], s[c + 3]);
+          mx2 = max3(mx2, s[c + 4], s[c + 5]);
+          mx3 = max3(mx3, s[c + 6], s[c + 7]);
+        }
+        const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+        // lazy rescale: keep the reference max unless the row max rose by more than 2^8
+        const bool grow = (m_ref == -INFINITY) ? (mt > -INFINITY) : (mt > m_ref + kRescale);
+        // O and the P buffer are both free once the PV of the previous tile is done
+        if (g >= 1 && !wait_pv(g - 1)) { ok = false; break; }
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          // O holds PV of the tiles before j: scale the rows that grow
+          tc_fence_after();
+          const float f = grow ? ex2(m_ref - mt) : 1.f;  // m_ref = -inf: O is still 0, f = 0
+          uint32_t o0[32], o1[32];
+          tmem_ld32_sync(o_tmem, o0);
+          tmem_ld32_sync(o_tmem + 32, o1);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            o0[c] = __float_as_uint(__uint_as_float(o0[c]) * f);
+            o1[c] = __float_as_uint(__uint_as_float(o1[c]) * f);
+          }
+          tmem_st32_sync(o_tmem, o0);
+          tmem_st32_sync(o_tmem + 32, o1);
+          l_run *= f;
+        }
+        if (grow) m_ref = mt;
+        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        const float2 sl2x2 = make_float2(sl2, sl2), negm = make_float2(-m_use, -m_use);
+        float2 sum0 = make_float2(0.f, 0.f), sum1 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < kBN / 32; ++q) {
+          // a 32-column chunk outside every lane's [lo, hi) needs no exponentials
+          const bool need = __any_sync(0xffffffffu, lo < q * 32 + 32 && hi > q * 32);
+          uint32_t pk[16];
+          if (need) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 4) {
+              float2 e0 = ffma2(make_float2(s[q * 32 + c], s[q * 32 + c + 1]), sl2x2, negm);
+              float2 e1 = ffma2(make_float2(s[q * 32 + c + 2], s[q * 32 + c + 3]), sl2x2, negm);
+              e0 = make_float2(ex2(e0.x), ex2(e0.y));
+              e1 = make_float2(ex2(e1.x), ex2(e1.y));
+              sum0 = fadd2(sum0, e0);
+              sum1 = fadd2(sum1, e1);
+              pk[c / 2] = pack_bf16x2(e0.x, e0.y);
+              pk[c / 2 + 1] = pack_bf16x2(e1.x, e1.y);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) pk[c] = 0u;
+          }
+          // P row -> shared memory, 128-byte swizzled K-major layout (16-byte chunk c of row r at c ^ (r & 7))
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int cc = q * 4 + u;  // 16-byte chunk index within the 128-byte row
+            *reinterpret_cast<uint4*>(prow + ((cc ^ sw) << 4)) =
+                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+          }
+        }
+        const float2 sum2 = fadd2(sum0, sum1);
+        l_run += sum2.x + sum2.y;
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full[sb]);
+      }
+      if (!ok) break;
+      // epilogue: the item's last PV, then O / l from TMEM
+      if (!wait_pv(g - 1)) { ok = false; break; }
       tc_fence_after();
       uint32_t o0[32], o1[32];
-      tmem_ld32_sync(lane_base + kOCol + ob * kDH, o0);
-      tmem_ld32_sync(lane_base + kOCol + ob * kDH + 32, o1);
+      tmem_ld32_sync(o_tmem, o0);
+      tmem_ld32_sync(o_tmem + 32, o1);
       tc_fence_before();
       mbar_arrive(&bars->o_empty[ob]);
-      const float f = acc_empty ? 0.f : ex2(m_acc_use - m_ref);
+      ++wi;
+      if (row_ok) {
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        uint4* dst = reinterpret_cast<uint4*>(O + ((tok0 + i) * H + it.h) * kDH);
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        acc[c] = fmaf(acc[c], f, __uint_as_float(o0[c]));
-        acc[c + 32] = fmaf(acc[c + 32], f, __uint_as_float(o1[c]));
+        for (int c = 0; c < 4; ++c) {
+          uint4 pk;
+          pk.x = pack_bf16x2(__uint_as_float(o0[c * 8 + 0]) * inv, __uint_as_float(o0[c * 8 + 1]) * inv);
+          pk.y = pack_bf16x2(__uint_as_float(o0[c * 8 + 2]) * inv, __uint_as_float(o0[c * 8 + 3]) * inv);
+          pk.z = pack_bf16x2(__uint_as_float(o0[c * 8 + 4]) * inv, __uint_as_float(o0[c * 8 + 5]) * inv);
+          pk.w = pack_bf16x2(__uint_as_float(o0[c * 8 + 6]) * inv, __uint_as_float(o0[c * 8 + 7]) * inv);
+          dst[c] = pk;
+          pk.x = pack_bf16x2(__uint_as_float(o1[c * 8 + 0]) * inv, __uint_as_float(o1[c * 8 + 1]) * inv);
+          pk.y = pack_bf16x2(__uint_as_float(o1[c * 8 + 2]) * inv, __uint_as_float(o1[c * 8 + 3]) * inv);
+          pk.z = pack_bf16x2(__uint_as_float(o1[c * 8 + 4]) * inv, __uint_as_float(o1[c * 8 + 5]) * inv);
+          pk.w = pack_bf16x2(__uint_as_float(o1[c * 8 + 6]) * inv, __uint_as_float(o1[c * 8 + 7]) * inv);
+          dst[4 + c] = pk;
+        }
+        if (a.lse)
+          a.lse[((int64_t)it.b * H + it.h) * n + i] = l_run > 0.f ? (m_ref + __log2f(l_run)) * kLn2 : -INFINITY;
       }
-      m_acc_use = m_ref;
-      acc_empty = false;
-      return true;
-    };
-
-    for (int j = 0; j < NT; ++j) {
-      const int sb = j & 1;
-      int lo, hi;
-      if (j < nbt) {
-        lo = 0;
-        hi = min(max(my_nbb - j * kBN, 0), kBN);
-      } else {
-        const int j0 = ls_first + (j - nbt) * kBN;
-        lo = min(max(my_ls - j0, 0), kBN);
-        hi = min(max(i - j0 + 1, 0), kBN);
-      }
-      if (!row_ok) { lo = 0; hi = 0; }
-      if (!mbar_wait_bounded(&bars->s_full[sb], (j >> 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
-      tc_fence_after();
-      float s[kBN];
-#pragma unroll
-      for (int q = 0; q < kBN / 32; ++q) {
-        uint32_t v[32];
-        tmem_ld32_sync(lane_base + kSCol + sb * kBN + q * 32, v);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) s[q * 32 + c] = __uint_as_float(v[c]);
-      }
-      float mt = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kBN; ++c) {
-        const float v = (c >= lo && c < hi) ? s[c] * sl2 : -INFINITY;
-        s[c] = v;
-        mt = fmaxf(mt, v);
-      }
-      const float m_new = fmaxf(m_run, mt);
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = ex2(m_run - m_use);  // 0 while nothing was seen
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < kBN; ++c) {
-        s[c] = ex2(s[c] - m_use);
-        sum += s[c];
-      }
-      l_run = l_run * alpha + sum;
-      m_run = m_new;
-      // P row -> shared memory, 128-byte swizzled K-major layout (16-byte chunk c of row r at c ^ (r & 7))
-      uint8_t* prow = p_row_base + sb * kPBytes;
-#pragma unroll
-      for (int cc = 0; cc < kBN / 8; ++cc) {
-        uint4 pk;
-        pk.x = pack_bf16x2(s[cc * 8 + 0], s[cc * 8 + 1]);
-        pk.y = pack_bf16x2(s[cc * 8 + 2], s[cc * 8 + 3]);
-        pk.z = pack_bf16x2(s[cc * 8 + 4], s[cc * 8 + 5]);
-        pk.w = pack_bf16x2(s[cc * 8 + 6], s[cc * 8 + 7]);
-        *reinterpret_cast<uint4*>(prow + (cc >> 3) * kTileBytes + (((cc & 7) ^ sw) << 4)) = pk;
-      }
-      fence_async_smem();
-      tc_fence_before();
-      mbar_arrive(&bars->p_full[sb]);
-      if (j >= 1 && !accumulate(j - 1, m_tile_use)) { ok = false; break; }
-      m_tile_use = m_use;
     }
-    if (ok) ok = accumulate(NT - 1, m_tile_use);
     if (!ok) {
       *abort_flag = 1;
       raise_status(a.status, ATTAMBA_DEV_TIMEOUT);
-    } else if (row_ok) {
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      uint4* dst = reinterpret_cast<uint4*>(O + ((tok0 + i) * H + h) * kDH);
-#pragma unroll
-      for (int c = 0; c < kDH / 8; ++c) {
-        uint4 pk;
-        pk.x = pack_bf16x2(acc[c * 8 + 0] * inv, acc[c * 8 + 1] * inv);
-        pk.y = pack_bf16x2(acc[c * 8 + 2] * inv, acc[c * 8 + 3] * inv);
-        pk.z = pack_bf16x2(acc[c * 8 + 4] * inv, acc[c * 8 + 5] * inv);
-        pk.w = pack_bf16x2(acc[c * 8 + 6] * inv, acc[c * 8 + 7] * inv);
-        dst[c] = pk;
-      }
-      if (a.lse)
-        a.lse[((int64_t)b * H + h) * n + i] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
     }
   }
 
@@ -395,13 +571,13 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
   return fn;
 }
 
-// [rows, H, 64] bf16 viewed as a 3-D tensor; box = 64 x 1 x 128 with the 128-byte swizzle
-bool encode_rows_map(CUtensorMap* m, const void* base, int64_t rows, int H) {
+// [rows, H, 64] bf16 viewed as a 3-D tensor; box = 64 x 1 x box_rows with the 128-byte swizzle
+bool encode_rows_map(CUtensorMap* m, const void* base, int64_t rows, int H, int box_rows) {
   auto enc = get_encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)kDH, (cuuint64_t)H, (cuuint64_t)rows};
   cuuint64_t strides[2] = {(cuuint64_t)kDH * 2, (cuuint64_t)H * kDH * 2};
-  cuuint32_t box[3] = {(cuuint32_t)kDH, 1, (cuuint32_t)kBN};
+  cuuint32_t box[3] = {(cuuint32_t)kDH, 1, (cuuint32_t)box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -413,9 +589,9 @@ bool encode_rows_map(CUtensorMap* m, const void* base, int64_t rows, int H) {
 cudaError_t launch_chunk_attn_bf16(const AttnArgs& a, cudaStream_t s) {
   const int64_t T = (int64_t)a.B * a.n;
   CUtensorMap tq, tk, tv, tkc, tvc;
-  if (!encode_rows_map(&tq, a.q, T, a.H) || !encode_rows_map(&tk, a.K, T, a.H) ||
-      !encode_rows_map(&tv, a.V, T, a.H) || !encode_rows_map(&tkc, a.Kc, a.n_chunks, a.H) ||
-      !encode_rows_map(&tvc, a.Vc, a.n_chunks, a.H))
+  if (!encode_rows_map(&tq, a.q, T, a.H, kBM) || !encode_rows_map(&tk, a.K, T, a.H, kBN) ||
+      !encode_rows_map(&tv, a.V, T, a.H, kBN) || !encode_rows_map(&tkc, a.Kc, a.n_chunks, a.H, kBN) ||
+      !encode_rows_map(&tvc, a.Vc, a.n_chunks, a.H, kBN))
     return cudaErrorNotSupported;
   static bool attr_set = false;
   if (!attr_set) {
@@ -424,8 +600,20 @@ cudaError_t launch_chunk_attn_bf16(const AttnArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid((a.n + kBM - 1) / kBM, a.H, a.B);
-  chunk_attn_bf16_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tkc, tvc, a);
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  // persistent: one CTA per SM, each walking the work items (sequence, head, 128 queries) round robin;
+  // more CTAs only when an SM would hold more items than its table
+  const int64_t items = (int64_t)((a.n + kBM - 1) / kBM) * a.B * a.H;
+  int64_t grid = items < (int64_t)kCtasPerSm * sms ? items : (int64_t)kCtasPerSm * sms;
+  if ((items + grid - 1) / grid > kMaxItems) grid = (items + kMaxItems - 1) / kMaxItems;
+  if (grid > 2147483647) return cudaErrorInvalidValue;
+  chunk_attn_bf16_kernel<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tkc, tvc, a);
   return cudaGetLastError();
 }
 

@@ -9,118 +9,311 @@
 //             h[d,:] = exp(delta A[d,:]) h[d,:] + delta x[t,d] B[t,:];
 //             y[t,d] = C[t,:] . h[d,:].
 //
-// Mapping (B200): chunks are independent, so the grid runs over
-// (channel pairs, groups of chunks, SSM) and every thread walks the tokens of
-// its chunk group for two channels, holding the 2 x N state and the 2 x N
-// decay rates (A * log2 e) in registers.  B and C, shared by all channels of a
-// token, are staged once per block in shared memory as fp32 and read as
-// broadcasts.  x and dt are read as packed pairs, coalesced across the warp.
-// The only global writes are the outputs (and the compact chunk-end rows).
-// The cost is set by the N exponentials per (token, channel, SSM), not by HBM.
+// Mapping (B200).  Chunks are independent, so the grid runs over (channel
+// groups, groups of chunks, SSM) and each thread walks the tokens of its chunk
+// group for CPT channels, holding the CPT x N state and the decay rates
+// (A * log2 e) in registers as f32x2 pairs over the state index, so the four
+// multiply-adds per element issue as two-wide instructions.  B and C, shared
+// by all channels of a token, are staged per block in shared memory as fp32 and
+// read as broadcast 16-byte loads.  x and dt of the next token are loaded while
+// the current one is computed.  The only global writes are the outputs.
+//
+// The work is one exponential per (token, channel, state, SSM): 2 T D N of them
+// against 10 D bytes per token, so the multi-function unit (16 ex2 per clock
+// per SM), not HBM, sets the pace.  For bf16 outputs a share of the
+// exponentials (kPolyPairs of the N/2 pairs) runs on the FMA pipe instead:
+// 2^x = 2^j * 2^f with j = round(x) (added to the exponent field) and 2^f from
+// a degree-3 polynomial fitted here by the Remez exchange algorithm to the
+// minimax relative error on [-1/2, 1/2] (max relative error 7.5e-5, far below
+// bf16's 2^-8).  The reduction is valid for x >= -125; a token where any lane
+// could go below uses the hardware exponential for every pair.  fp32 outputs
+// use the hardware exponential only.
 #include "common.cuh"
 #include "launch.h"
+
+#ifndef ATTAMBA_SCAN_POLY_PAIRS
+#define ATTAMBA_SCAN_POLY_PAIRS 0
+#endif
+#ifndef ATTAMBA_SCAN_CPT
+#define ATTAMBA_SCAN_CPT 2
+#endif
+#ifndef ATTAMBA_SCAN_MINB
+#define ATTAMBA_SCAN_MINB 4
+#endif
 
 namespace attamba {
 
 namespace {
 constexpr int kScanThreads = 128;
-constexpr int kStageTokens = 32;
+constexpr int kStageTokens = 64;
+constexpr int kMaxChunksPerBlock = 64;
+constexpr int kNS = 16;
+constexpr int kNP = kNS / 2;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kPolyMinExp = -125.f;
+// 2^f on [-1/2, 1/2], minimax relative error (own Remez fit), f32 coefficients
+constexpr float kP0 = 0.9999280571937561f;
+constexpr float kP1 = 0.6932609677314758f;
+constexpr float kP2 = 0.2426111251115799f;
+constexpr float kP3 = 0.0551716685295105f;
 
-__device__ __forceinline__ float softplus_f(float z) {
-  return z > 20.f ? z : log1pf(__expf(z));
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(reinterpret_cast<uint64_t&>(d))
+      : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)),
+        "l"(reinterpret_cast<const uint64_t&>(c)));
+  return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;"
+      : "=l"(reinterpret_cast<uint64_t&>(d))
+      : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)));
+  return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("add.rn.f32x2 %0, %1, %2;"
+      : "=l"(reinterpret_cast<uint64_t&>(d))
+      : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)));
+  return d;
 }
 
-template <typename T, int NS>
-__global__ void __launch_bounds__(kScanThreads) kv_ssm_scan_kernel(ScanArgs p, int32_t chunks_per_block) {
-  __shared__ __align__(16) float sB[kStageTokens][NS];
-  __shared__ __align__(16) float sC[kStageTokens][NS];
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  float2 d;
+  asm("sub.rn.f32x2 %0, %1, %2;"
+      : "=l"(reinterpret_cast<uint64_t&>(d))
+      : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)));
+  return d;
+}
+
+// 2^x for x in [-125, 0] on the FMA pipe (see the file comment)
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  const float2 magic = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23: x + magic rounds x to an integer
+  const float2 t = add2(x, magic);
+  const float2 j = add2(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = sub2(x, j);
+  float2 p = fma2(f, make_float2(kP3, kP3), make_float2(kP2, kP2));
+  p = fma2(p, f, make_float2(kP1, kP1));
+  p = fma2(p, f, make_float2(kP0, kP0));
+  // the low mantissa bits of t hold j; shifted into the exponent field they scale p by 2^j
+  return make_float2(__uint_as_float(__float_as_uint(t.x) * 8388608u + __float_as_uint(p.x)),
+                     __uint_as_float(__float_as_uint(t.y) * 8388608u + __float_as_uint(p.y)));
+}
+
+// softplus(z) = log(1 + e^z) with u = e^z:  log2(1 + u) on the multi-function unit
+// when u >= 1/16 (its absolute error, about 2^-22, is then below 3e-6 of the
+// result), the series u - u^2/2 + u^3/3 - u^4/4 + u^5/5 below (truncation under
+// u^5/6 relative), and z itself above 20.
+__device__ __forceinline__ float softplus_f(float z) {
+  const float u = ex2(z * kLog2e);
+  float lg;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(1.f + u));
+  const float ser = u * fmaf(u, fmaf(u, fmaf(u, fmaf(u, 0.2f, -0.25f), 1.f / 3.f), -0.5f), 1.f);
+  const float v = u < 0.0625f ? ser : lg * 0.6931471805599453f;
+  return z > 20.f ? z : v;
+}
+
+template <typename T, int CPT> struct Vec;
+template <> struct Vec<__nv_bfloat16, 2> {
+  using raw = uint32_t;
+  static __device__ __forceinline__ raw load(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint32_t*>(p)); }
+  static __device__ __forceinline__ void unpack(raw r, float (&v)[2]) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r));
+    v[0] = f.x; v[1] = f.y;
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[2]) {
+    *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v[0], v[1]);
+  }
+};
+template <> struct Vec<__nv_bfloat16, 4> {
+  using raw = uint2;
+  static __device__ __forceinline__ raw load(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint2*>(p)); }
+  static __device__ __forceinline__ void unpack(raw r, float (&v)[4]) {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[4]) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
+    uint2 r;
+    r.x = *reinterpret_cast<uint32_t*>(&a);
+    r.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = r;
+  }
+};
+template <> struct Vec<float, 4> {
+  using raw = float4;
+  static __device__ __forceinline__ raw load(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+  static __device__ __forceinline__ void unpack(raw r, float (&v)[4]) { v[0] = r.x; v[1] = r.y; v[2] = r.z; v[3] = r.w; }
+  static __device__ __forceinline__ void store(float* p, const float (&v)[4]) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+};
+template <> struct Vec<float, 2> {
+  using raw = float2;
+  static __device__ __forceinline__ raw load(const float* p) { return __ldg(reinterpret_cast<const float2*>(p)); }
+  static __device__ __forceinline__ void unpack(raw r, float (&v)[2]) { v[0] = r.x; v[1] = r.y; }
+  static __device__ __forceinline__ void store(float* p, const float (&v)[2]) {
+    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+  }
+};
+
+// Per-thread state of the scan: CPT channels x N/2 state pairs.
+template <int CPT> struct ScanState {
+  float2 a2[CPT][kNP];  // A * log2 e
+  float2 h[CPT][kNP];
+  float bias[CPT];
+  float amax;           // largest |A| log2 e of the thread's channels
+};
+
+// One token: decay, input, readout.  `reset` marks a chunk start: its delta in
+// the exponent is replaced by a huge value so exp(delta A) = 0 (A < 0) and the
+// state restarts from the token's own input, with no branch.
+template <typename T, int CPT, int POLY_PAIRS>
+__device__ __forceinline__ void scan_token(ScanState<CPT>& st, const float* __restrict__ bc, const float (&dl)[CPT],
+                                           const float (&dx)[CPT], bool reset, bool poly_ok, float (&y)[CPT]) {
+  const float4* bc4 = reinterpret_cast<const float4*>(bc);
+  float2 Bp[kNP], Cp[kNP];
+#pragma unroll
+  for (int q = 0; q < kNP / 2; ++q) {
+    const float4 b4 = bc4[q], c4 = bc4[kNP / 2 + q];
+    Bp[2 * q] = make_float2(b4.x, b4.y);
+    Bp[2 * q + 1] = make_float2(b4.z, b4.w);
+    Cp[2 * q] = make_float2(c4.x, c4.y);
+    Cp[2 * q + 1] = make_float2(c4.z, c4.w);
+  }
+#pragma unroll
+  for (int cc = 0; cc < CPT; ++cc) {
+    const float de = reset ? 1e30f : dl[cc];
+    const float2 dl2 = make_float2(de, de);
+    const float2 dx2 = make_float2(dx[cc], dx[cc]);
+    float2 ya = make_float2(0.f, 0.f), yb = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < kNP; ++q) {
+      const float2 e = mul2(dl2, st.a2[cc][q]);
+      float2 a;
+      if (q < POLY_PAIRS && poly_ok) a = exp2_poly2(e);
+      else a = make_float2(ex2(e.x), ex2(e.y));
+      st.h[cc][q] = fma2(a, st.h[cc][q], mul2(dx2, Bp[q]));
+      if (q & 1) yb = fma2(Cp[q], st.h[cc][q], yb);
+      else ya = fma2(Cp[q], st.h[cc][q], ya);
+    }
+    y[cc] = (ya.x + ya.y) + (yb.x + yb.y);
+  }
+}
+
+template <typename T, int CPT, int POLY_PAIRS>
+__global__ void __launch_bounds__(kScanThreads, ATTAMBA_SCAN_MINB) kv_ssm_scan_kernel(ScanArgs p, int32_t chunks_per_block) {
+  using V = Vec<T, CPT>;
+  __shared__ __align__(16) float sBC[kStageTokens][2 * kNS];  // B then C of each staged token
+  __shared__ int sCu[kMaxChunksPerBlock + 1];                 // chunk starts of this block
 
   const int s = blockIdx.z;
-  const int D = p.D;
-  const int d0 = (blockIdx.x * kScanThreads + threadIdx.x) * 2;
+  const int D = p.D;  // T * D < 2^31 (checked by the host): 32-bit element offsets
+  const int d0 = (blockIdx.x * kScanThreads + threadIdx.x) * CPT;
   const bool active = d0 < D;
   const int32_t c_begin = blockIdx.y * chunks_per_block;
   if (c_begin >= p.n_chunks) return;
   const int32_t c_end = min(c_begin + chunks_per_block, p.n_chunks);
+  for (int i = threadIdx.x; i <= c_end - c_begin; i += kScanThreads) sCu[i] = p.cu[c_begin + i];
 
-  const T* __restrict__ x = static_cast<const T*>(p.x);
-  const T* __restrict__ dt = static_cast<const T*>(p.dt[s]);
+  const T* __restrict__ x = static_cast<const T*>(p.x) + d0;
+  const T* __restrict__ dt = static_cast<const T*>(p.dt[s]) + d0;
   const T* __restrict__ Bm = static_cast<const T*>(p.Bm[s]);
   const T* __restrict__ Cm = static_cast<const T*>(p.Cm[s]);
-  T* __restrict__ out = static_cast<T*>(p.out[s]);
+  T* __restrict__ out = static_cast<T*>(p.out[s]) + d0;
   T* __restrict__ outc = static_cast<T*>(p.outc[s]);
-  const int32_t* __restrict__ cu = p.cu;
 
-  float a2[2][NS];
-  float bias[2] = {0.f, 0.f};
-  float h[2][NS];
+  ScanState<CPT> st;
+  st.amax = 0.f;
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
+  for (int c = 0; c < CPT; ++c) {
+    st.bias[c] = active ? p.bias[s][d0 + c] : 0.f;
 #pragma unroll
-    for (int n = 0; n < NS; ++n) {
-      a2[j][n] = active ? p.A[s][(size_t)(d0 + j) * NS + n] * kLog2e : 0.f;
-      h[j][n] = 0.f;
+    for (int q = 0; q < kNP; ++q) {
+      float2 v = make_float2(0.f, 0.f);
+      if (active) v = *reinterpret_cast<const float2*>(p.A[s] + (size_t)(d0 + c) * kNS + 2 * q);
+      st.a2[c][q] = make_float2(v.x * kLog2e, v.y * kLog2e);
+      st.amax = fmaxf(st.amax, fmaxf(-st.a2[c][q].x, -st.a2[c][q].y));
+      st.h[c][q] = make_float2(0.f, 0.f);
     }
-    if (active) bias[j] = p.bias[s][d0 + j];
   }
+  __syncthreads();
+  const int t_begin = sCu[0];
+  const int t_end = sCu[c_end - c_begin];
+  int ci = 0;                 // chunk of the current token, relative to c_begin
+  int next_start = sCu[1];
 
-  const int64_t t_begin = cu[c_begin];
-  const int64_t t_end = cu[c_end];
-  int32_t c = c_begin;
-  int64_t next_start = cu[c + 1];
+  // delta of the next token, computed one token ahead from loads issued one token ahead
+  float dl_n[CPT], dx_n[CPT];
+  auto delta_of = [&](typename V::raw xr, typename V::raw zr) {
+    float xv[CPT], zv[CPT];
+    V::unpack(xr, xv);
+    V::unpack(zr, zv);
+#pragma unroll
+    for (int cc = 0; cc < CPT; ++cc) {
+      dl_n[cc] = softplus_f(zv[cc] + st.bias[cc]);
+      dx_n[cc] = dl_n[cc] * xv[cc];
+    }
+  };
+  if (active) delta_of(V::load(x + t_begin * D), V::load(dt + t_begin * D));
 
-  for (int64_t tb = t_begin; tb < t_end; tb += kStageTokens) {
-    const int nt = (int)((t_end - tb) < kStageTokens ? (t_end - tb) : kStageTokens);
-    __syncthreads();
-    for (int e = threadIdx.x; e < nt * NS; e += kScanThreads) {
-      const int k = e / NS, n = e - k * NS;
-      sB[k][n] = Elem<T>::to_f(Bm[(tb + k) * NS + n]);
-      sC[k][n] = Elem<T>::to_f(Cm[(tb + k) * NS + n]);
+  auto step = [&](int t, const float* bc) {
+    const int tn = min(t + 1, t_end - 1);  // the next token (clamped: a harmless reload at the end)
+    const typename V::raw xr = V::load(x + tn * D), zr = V::load(dt + tn * D);
+    float dl[CPT], dx[CPT], dmax = 0.f;
+#pragma unroll
+    for (int cc = 0; cc < CPT; ++cc) {
+      dl[cc] = dl_n[cc];
+      dx[cc] = dx_n[cc];
+      dmax = fmaxf(dmax, dl[cc]);
+    }
+    const bool reset = (t == next_start);
+    ci += reset ? 1 : 0;
+    next_start = sCu[ci + 1];
+    bool poly_ok = false;
+    if (POLY_PAIRS > 0) poly_ok = !reset && !__any_sync(__activemask(), dmax * st.amax > -kPolyMinExp);
+    float y[CPT];
+    scan_token<T, CPT, POLY_PAIRS>(st, bc, dl, dx, reset, poly_ok, y);
+    V::store(out + t * D, y);
+    if (outc != nullptr && t + 1 == next_start) V::store(outc + (c_begin + ci) * D + d0, y);
+    delta_of(xr, zr);
+  };
+
+  for (int tb = t_begin; tb < t_end; tb += kStageTokens) {
+    const int nt = min(kStageTokens, t_end - tb);
+    if (tb != t_begin) __syncthreads();
+    for (int e = threadIdx.x; e < nt * kNS; e += kScanThreads) {
+      const int k = e / kNS, n = e - k * kNS;
+      sBC[k][n] = Elem<T>::to_f(Bm[(tb + k) * kNS + n]);
+      sBC[k][kNS + n] = Elem<T>::to_f(Cm[(tb + k) * kNS + n]);
     }
     __syncthreads();
     if (!active) continue;
-    for (int k = 0; k < nt; ++k) {
-      const int64_t t = tb + k;
-      if (t == next_start) {  // a new chunk: restart the state
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-          for (int n = 0; n < NS; ++n) h[j][n] = 0.f;
-        ++c;
-        next_start = cu[c + 1];
-      }
-      const float2 xv = load2(x + t * D + d0);
-      const float2 zv = load2(dt + t * D + d0);
-      const float dl0 = softplus_f(zv.x + bias[0]);
-      const float dl1 = softplus_f(zv.y + bias[1]);
-      const float dx0 = dl0 * xv.x, dx1 = dl1 * xv.y;
-      float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-      for (int n = 0; n < NS; ++n) {
-        const float bn = sB[k][n], cn = sC[k][n];
-        h[0][n] = fmaf(ex2(dl0 * a2[0][n]), h[0][n], dx0 * bn);
-        h[1][n] = fmaf(ex2(dl1 * a2[1][n]), h[1][n], dx1 * bn);
-        y0 = fmaf(cn, h[0][n], y0);
-        y1 = fmaf(cn, h[1][n], y1);
-      }
-      store2(out + t * D + d0, y0, y1);
-      if (outc != nullptr && t + 1 == next_start) store2(outc + (int64_t)c * D + d0, y0, y1);
+    int k = 0;
+    for (; k + 1 < nt; k += 2) {  // two tokens per iteration: their independent work interleaves
+      step(tb + k, &sBC[k][0]);
+      step(tb + k + 1, &sBC[k + 1][0]);
     }
+    if (k < nt) step(tb + k, &sBC[k][0]);
   }
 }
 }  // namespace
 
 cudaError_t launch_kv_ssm_scan(attamba_dtype_t dtype, const ScanArgs& a, cudaStream_t s) {
+  constexpr int CPT = ATTAMBA_SCAN_CPT;
   // about 64 tokens of chunks per block
   int64_t cpb = (64 * (int64_t)a.n_chunks) / (a.T > 0 ? a.T : 1);
   if (cpb < 1) cpb = 1;
-  while ((a.n_chunks + cpb - 1) / cpb > 65535) cpb *= 2;
-  dim3 grid((a.D / 2 + kScanThreads - 1) / kScanThreads, (unsigned)((a.n_chunks + cpb - 1) / cpb), 2);
+  if (cpb > kMaxChunksPerBlock) cpb = kMaxChunksPerBlock;
+  if ((a.n_chunks + cpb - 1) / cpb > 65535) return cudaErrorInvalidValue;
+  dim3 grid((a.D / CPT + kScanThreads - 1) / kScanThreads, (unsigned)((a.n_chunks + cpb - 1) / cpb), 2);
   if (dtype == ATTAMBA_BF16)
-    kv_ssm_scan_kernel<__nv_bfloat16, 16><<<grid, kScanThreads, 0, s>>>(a, (int32_t)cpb);
+    kv_ssm_scan_kernel<__nv_bfloat16, CPT, ATTAMBA_SCAN_POLY_PAIRS><<<grid, kScanThreads, 0, s>>>(a, (int32_t)cpb);
   else
-    kv_ssm_scan_kernel<float, 16><<<grid, kScanThreads, 0, s>>>(a, (int32_t)cpb);
+    kv_ssm_scan_kernel<float, CPT, 0><<<grid, kScanThreads, 0, s>>>(a, (int32_t)cpb);
   return cudaGetLastError();
 }
 

@@ -10,7 +10,8 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import assert_close, f64, oracle_attention_seq, oracle_scan_seq, run_prefill
+from helpers import (assert_close, attn_rounding_bound, f64, key_lists, oracle_attention_seq, oracle_scan_seq,
+                     run_prefill)
 from ssm_compressed_chunked_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -55,9 +56,11 @@ def test_attention_small(cfg):
         assert_close(cfg.dtype, lse[b][fin], rl[fin], f"lse b={b}")
         # end to end: oracle scan + oracle attention
         rk, rv = oracle_scan_seq(inp, b)
-        eo, _ = oracle_attention_seq(q, rk.reshape(n, H, dh), rv.reshape(n, H, dh), st, n, cfg.L, cfg.mode,
-                                     inp["scale"])
-        assert_close(cfg.dtype, f64(O[b]), eo, f"O (end to end) b={b}")
+        rk, rv = rk.reshape(n, H, dh), rv.reshape(n, H, dh)
+        eo, _ = oracle_attention_seq(q, rk, rv, st, n, cfg.L, cfg.mode, inp["scale"])
+        extra = 0.0 if cfg.dtype == "f32" else attn_rounding_bound(
+            q, rk, rv, eo, key_lists(n, st, cfg.L, cfg.mode, range(n)), inp["scale"])
+        assert_close(cfg.dtype, f64(O[b]), eo, f"O (end to end) b={b}", extra=extra)
     assert pf.status.item() == 0
 
 
@@ -78,9 +81,10 @@ def test_attention_full_size_sampled_rows(cfg):
     ro, _ = oracle_attention_seq(q, f64(K[b]), f64(V[b]), st, n, cfg.L, cfg.mode, inp["scale"], rows)
     assert_close(cfg.dtype, f64(O[b])[rows], ro, "O (isolated, sampled)")
     rk, rv = oracle_scan_seq(inp, b)
-    eo, _ = oracle_attention_seq(q, rk.reshape(n, H, dh), rv.reshape(n, H, dh), st, n, cfg.L, cfg.mode,
-                                 inp["scale"], rows)
-    assert_close(cfg.dtype, f64(O[b])[rows], eo, "O (end to end, sampled)")
+    rk, rv = rk.reshape(n, H, dh), rv.reshape(n, H, dh)
+    eo, _ = oracle_attention_seq(q, rk, rv, st, n, cfg.L, cfg.mode, inp["scale"], rows)
+    extra = attn_rounding_bound(q[rows], rk, rv, eo, key_lists(n, st, cfg.L, cfg.mode, rows), inp["scale"])
+    assert_close(cfg.dtype, f64(O[b])[rows], eo, "O (end to end, sampled)", extra=extra)
     assert pf.status.item() == 0
 
 

@@ -1,0 +1,49 @@
+"""Host logic of the multi-GPU bench on CPU: two gloo ranks (no GPU, no collective on the data path)."""
+
+import os
+import socket
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, ws, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(ws), RANK=str(rank),
+                      LOCAL_RANK=str(rank))
+    import bench
+    w, r, _ = bench.setup_dist()
+    assert (w, r) == (ws, rank)
+    cfg = bench.rank_config(bench.CFG, w, r)
+    # each rank's step time differs; every rank must see the slowest one
+    mx = bench.max_over_ranks(1.0 + rank, w)
+    bench.barrier(w)
+    value = bench.job_throughput(w, cfg.B * cfg.n, mx)
+    out[rank] = (cfg.seed, mx, value)
+    import torch.distributed as dist
+    dist.destroy_process_group()
+
+
+def test_two_ranks_take_the_max_and_use_their_own_seeds():
+    ws = 2
+    out = mp.Manager().dict()
+    mp.spawn(_worker, args=(ws, _free_port(), out), nprocs=ws, join=True)
+    seeds = {out[r][0] for r in range(ws)}
+    assert len(seeds) == ws                       # distinct batches per rank (weak scaling)
+    assert all(out[r][1] == 2.0 for r in range(ws))   # max over ranks
+    import bench
+    T = bench.CFG.B * bench.CFG.n
+    assert all(abs(out[r][2] - ws * T / 2e-3) < 1e-6 for r in range(ws))
+
+
+def test_reference_arm_runs_on_rank_zero_only(capsys):
+    import argparse
+    import bench
+    bench.run_reference(argparse.Namespace(steps=1, warmup=0), 2, 1)   # rank 1: no work, no output
+    assert capsys.readouterr().out == ""
