@@ -188,6 +188,31 @@ attamba_status_t attamba_decode_step(attamba_dtype_t dtype, const attamba_cache_
                                      size_t workspace_bytes, int32_t* d_status,
                                      attamba_stream_t stream);
 
+/* attamba_decode_step_noalloc -- attamba_decode_step without a caller workspace.
+ * The paper has no counterpart to this entry point; it exists for callers that
+ * cannot allocate device memory when they step the decoder: hosts that hand out
+ * all device memory up front from their own pool and forbid cudaMalloc later
+ * (it may synchronize the device and can fail mid-stream), or callers that have
+ * no channel for passing this library a scratch buffer.
+ *   Same arguments and behaviour as attamba_decode_step, minus workspace and
+ *   workspace_bytes.  The split-K scratch is a fixed 4 MiB array inside the
+ *   library, allocated with the library's device code on each GPU that loads it
+ *   and kept until the process exits.  A cache needing more than that
+ *   (attamba_decode_workspace_size(cache) > 4 MiB) is rejected with
+ *   ATTAMBA_ERR_UNSUPPORTED before any launch; attamba_last_error() says so.
+ *   The first call on a device looks up the array's device address (no
+ *   allocation); make that first call before capturing a stream.
+ *   All calls on a device share the array and it keeps the last call's
+ *   contents (nothing in it needs to start at zero).  Calls whose kernels can
+ *   overlap on the GPU (unordered streams) race on it; order them on one stream. */
+attamba_status_t attamba_decode_step_noalloc(attamba_dtype_t dtype, const attamba_cache_t* cache,
+                                             const void* q_t, const void* x_t, const void* dt_k,
+                                             const void* dt_v, const float* bias_k, const float* bias_v,
+                                             const float* A_k, const float* A_v, const void* B_k,
+                                             const void* C_k, const void* B_v, const void* C_v,
+                                             float scale, void* o_t, int32_t* d_status,
+                                             attamba_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,7 +24,8 @@ DEV_BAD_CHUNKS, DEV_CACHE_FULL, DEV_TIMEOUT = 0x1, 0x2, 0x4
 # every symbol include/attamba.h declares
 EXPORTS = ("attamba_version", "attamba_status_string", "attamba_last_error",
            "attamba_uniform_chunk_count", "attamba_chunk_index", "attamba_kv_ssm_scan",
-           "attamba_chunk_attn_fwd", "attamba_decode_workspace_size", "attamba_decode_step")
+           "attamba_chunk_attn_fwd", "attamba_decode_workspace_size", "attamba_decode_step",
+           "attamba_decode_step_noalloc")
 
 
 class AttambaError(RuntimeError):
@@ -75,6 +76,8 @@ def load():
     L.attamba_decode_step.restype = ctypes.c_int
     L.attamba_decode_step.argtypes = [ctypes.c_int, ctypes.POINTER(CacheT)] + [vp] * 12 + \
                                      [f32, vp, vp, sz, vp, vp]
+    L.attamba_decode_step_noalloc.restype = ctypes.c_int
+    L.attamba_decode_step_noalloc.argtypes = [ctypes.c_int, ctypes.POINTER(CacheT)] + [vp] * 12 + [f32, vp, vp, vp]
     _lib = L
     return L
 
@@ -208,3 +211,18 @@ def decode_step(cache, q_t, x_t, dt_k, dt_v, bias_k, bias_v, A_k, A_v, B_k, C_k,
         _ptr(workspace, None, "workspace"), workspace.numel() * workspace.element_size(),
         _ptr(status, torch.int32, "status", allow_none=True), _stream(stream))
     _check(st, "attamba_decode_step")
+
+
+def decode_step_noalloc(cache, q_t, x_t, dt_k, dt_v, bias_k, bias_v, A_k, A_v, B_k, C_k, B_v, C_v, scale, o_t,
+                        status=None, stream=None):
+    """attamba_decode_step_noalloc: one decode step whose split-K scratch is the library's own
+    fixed device array, for callers that cannot allocate a workspace (see include/attamba.h)."""
+    dt = torch.bfloat16
+    f32 = torch.float32
+    st = load().attamba_decode_step_noalloc(
+        BF16, ctypes.byref(cache.c_struct()), _ptr(q_t, dt, "q_t"), _ptr(x_t, dt, "x_t"),
+        _ptr(dt_k, dt, "dt_k"), _ptr(dt_v, dt, "dt_v"), _ptr(bias_k, f32, "bias_k"), _ptr(bias_v, f32, "bias_v"),
+        _ptr(A_k, f32, "A_k"), _ptr(A_v, f32, "A_v"), _ptr(B_k, dt, "B_k"), _ptr(C_k, dt, "C_k"),
+        _ptr(B_v, dt, "B_v"), _ptr(C_v, dt, "C_v"), float(scale), _ptr(o_t, dt, "o_t"),
+        _ptr(status, torch.int32, "status", allow_none=True), _stream(stream))
+    _check(st, "attamba_decode_step_noalloc")

@@ -168,4 +168,52 @@ attamba_status_t attamba_decode_step(attamba_dtype_t dtype, const attamba_cache_
   return e == cudaSuccess ? ATTAMBA_OK : cuda_fail(e, "attamba_decode_step");
 }
 
+attamba_status_t attamba_decode_step_noalloc(attamba_dtype_t dtype, const attamba_cache_t* cache,
+                                             const void* q_t, const void* x_t, const void* dt_k,
+                                             const void* dt_v, const float* bias_k, const float* bias_v,
+                                             const float* A_k, const float* A_v, const void* B_k,
+                                             const void* C_k, const void* B_v, const void* C_v,
+                                             float scale, void* o_t, int32_t* d_status,
+                                             attamba_stream_t stream) {
+  if (dtype != ATTAMBA_BF16) return ATTAMBA_ERR_UNSUPPORTED;
+  if (!cache) return ATTAMBA_ERR_INVALID_ARG;
+  const attamba_cache_t& c = *cache;
+  if (c.dh != 64 || c.N != 16) return ATTAMBA_ERR_UNSUPPORTED;
+  if (c.B < 1 || c.H < 1 || c.P < 1 || c.L < 1 || c.cap < 1) return ATTAMBA_ERR_INVALID_ARG;
+  if ((int64_t)c.B * c.H * c.cap * c.dh >= ((int64_t)1 << 40)) return ATTAMBA_ERR_INVALID_ARG;
+  const void* req[] = {c.state, c.Kb, c.Vb, c.bpos, c.Kr, c.Vr, c.nb, c.pos, q_t, x_t, dt_k, dt_v,
+                       bias_k, bias_v, A_k, A_v, B_k, C_k, B_v, C_v, o_t};
+  for (const void* p : req)
+    if (!p) return ATTAMBA_ERR_INVALID_ARG;
+  const void* al[] = {c.Kb, c.Vb, c.Kr, c.Vr, q_t};
+  for (const void* p : al)
+    if (!aligned16(p)) return ATTAMBA_ERR_INVALID_ARG;
+  if (!(scale > 0.f)) return ATTAMBA_ERR_INVALID_ARG;
+  const size_t need = attamba::decode_workspace_bytes(c);
+  if (need > attamba::decode_noalloc_scratch_bytes()) {
+    snprintf(g_err, sizeof(g_err),
+             "attamba_decode_step_noalloc: this cache needs %zu bytes of split-K scratch, the built-in "
+             "scratch holds %zu; use attamba_decode_step with a workspace",
+             need, attamba::decode_noalloc_scratch_bytes());
+    return ATTAMBA_ERR_UNSUPPORTED;
+  }
+  float* scratch = nullptr;
+  cudaError_t e = attamba::decode_noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "attamba_decode_step_noalloc (scratch address)");
+  attamba::DecodeArgs a{};
+  a.c = c;
+  a.q = q_t; a.x = x_t;
+  a.dt[0] = dt_k; a.dt[1] = dt_v;
+  a.bias[0] = bias_k; a.bias[1] = bias_v;
+  a.A[0] = A_k; a.A[1] = A_v;
+  a.Bm[0] = B_k; a.Bm[1] = B_v;
+  a.Cm[0] = C_k; a.Cm[1] = C_v;
+  a.scale = scale; a.o = o_t;
+  a.work = scratch;
+  a.splits = attamba::decode_splits(c);
+  a.status = d_status;
+  e = attamba::launch_decode_step(a, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTAMBA_OK : cuda_fail(e, "attamba_decode_step_noalloc");
+}
+
 }  // extern "C"

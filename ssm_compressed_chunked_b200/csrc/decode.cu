@@ -19,10 +19,22 @@
 //   decode_combine_kernel per (sequence, head): merges the splits, writes o_t,
 //                         and advances pos / nb
 // The step is bound by streaming the cached K/V from HBM.
+#include <mutex>
+
 #include "common.cuh"
 #include "launch.h"
 
 namespace attamba {
+
+// Split-K scratch of attamba_decode_step_noalloc: a fixed array in the
+// library's own device memory, so that entry point never allocates.  It holds
+// B * H * splits * (head_dim + 2) floats of partial results; every (sequence,
+// head, split) slot is written by decode_attn_kernel before decode_combine_kernel
+// reads it, so nothing in it has to start at zero.  All calls on a device share
+// it: two no-alloc calls whose kernels overlap on the GPU (different streams,
+// no ordering between them) corrupt each other's partials.
+constexpr size_t kNoAllocScratchFloats = (size_t)1 << 20;  // 4 MiB
+static __device__ __align__(256) float g_decode_scratch[kNoAllocScratchFloats];
 
 namespace {
 constexpr int kDH = 64;
@@ -263,6 +275,29 @@ int32_t decode_splits(const attamba_cache_t& c) {
   if (sp > max_sp) sp = max_sp;
   if (sp < 1) sp = 1;
   return (int32_t)sp;
+}
+
+size_t decode_noalloc_scratch_bytes() { return kNoAllocScratchFloats * sizeof(float); }
+
+// Device address of g_decode_scratch on the current device.  The name is a host
+// stand-in, not a device pointer, so the address is asked of the runtime once
+// per device (with that device current) and cached.
+cudaError_t decode_noalloc_scratch(float** out) {
+  static std::mutex mu;
+  static float* cached[128] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    cached[dev] = static_cast<float*>(p);
+  }
+  *out = cached[dev];
+  return cudaSuccess;
 }
 
 size_t decode_workspace_bytes(const attamba_cache_t& c) {

@@ -67,6 +67,8 @@ struct DecodeArgs {
 };
 int32_t decode_splits(const attamba_cache_t& c);
 size_t decode_workspace_bytes(const attamba_cache_t& c);
+size_t decode_noalloc_scratch_bytes();
+cudaError_t decode_noalloc_scratch(float** out);
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s);
 
 }  // namespace attamba
