@@ -232,6 +232,53 @@ def cpu_baseline():
                       f"(float64 scan of K and V + dense M_test attention), {dt:.1f} s"}
 
 
+# ------------------------------------------------------------------ decode row
+def decode_bench(dev, reps=3):
+    """128 decode steps of the decode workload (B=32, 16384 compressed tokens of context, P=8, L=64):
+    tokens/s and the HBM fraction of the whole step (cached K/V read + SSM state read/write)."""
+    from ssm_compressed_chunked_b200 import attamba as A
+    cfg = W.DECODE_CONFIG
+    dec = W.make_decode(cfg)
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in dec.items()}
+    names = ("state", "Kb", "Vb", "bpos", "Kr", "Vr", "nbuf", "pos")
+    work = {k: g[k].clone() for k in names}
+    cache = A.Cache(work["state"], work["Kb"], work["Vb"], work["bpos"], work["Kr"], work["Vr"], work["nbuf"],
+                    work["pos"], cfg.P, cfg.offset)
+    ws_buf = torch.empty(A.decode_workspace_size(cache), dtype=torch.uint8, device=dev)
+    o = torch.empty(cfg.B, cfg.H, cfg.dh, dtype=torch.bfloat16, device=dev)
+
+    def steps():
+        for st in range(cfg.steps):
+            A.decode_step(cache, g["q"][st], g["x"][st], g["dt_k"][st], g["dt_v"][st], g["bias_k"], g["bias_v"],
+                          g["A_k"], g["A_v"], g["B_k"][st], g["C_k"][st], g["B_v"][st], g["C_v"][st], dec["scale"],
+                          o, ws_buf)
+
+    times = []
+    for rep in range(reps + 1):
+        for k in names:
+            work[k].copy_(g[k])
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        steps()
+        e1.record()
+        torch.cuda.synchronize()
+        if rep > 0:
+            times.append(e0.elapsed_time(e1))
+    ms = float(np.median(times))
+    # keys read per step: chunk ends below the window plus the window, for t = ctx .. ctx + steps - 1
+    keys = sum((t - cfg.L + 1) // cfg.P + cfg.L for t in range(cfg.ctx, cfg.ctx + cfg.steps)) / cfg.steps
+    D = cfg.H * cfg.dh
+    step_bytes = cfg.B * cfg.H * keys * cfg.dh * 2 * 2 + 2 * 2 * cfg.B * cfg.N * D * 4
+    hbm, _, _, src = peaks()
+    per_step = ms / cfg.steps
+    gbs = step_bytes / (per_step * 1e-3) / 1e9
+    return {"workload": cfg.name, "tokens_per_s": cfg.B * cfg.steps / (ms * 1e-3), "ms_per_step": per_step,
+            "steps": cfg.steps, "batch": cfg.B, "context": cfg.ctx, "bytes_per_step": step_bytes,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "peak_source": f"{src} HBM copy"}, "gpu_launches_per_step": 3}
+
+
 # ------------------------------------------------------------------ CUDA path
 def run_ours(args, ws, rank, local):
     from ssm_compressed_chunked_b200 import attamba as A, layer
@@ -342,7 +389,14 @@ def run_ours(args, ws, rank, local):
         d["share"] = d["ms"] / mean.sum()
     dom = max(kernels, key=lambda k: kernels[k]["ms"])
     d = kernels[dom]
-    if dom == "chunk_attn_fwd":
+    exp_peak = 16 * 148 * 1.965e9  # ex2 per second: 16 per clock per SM, 148 SMs, 1965 MHz
+    if dom == "kv_ssm_scan":
+        ach = d["exps"] / (d["ms"] * 1e-3) / 1e9
+        roof = {"bound": "alu", "achieved": ach, "peak": exp_peak / 1e9, "unit": "Gexp/s", "frac": ach / (exp_peak / 1e9),
+                "peak_source": "multi-function unit: 16 ex2/clk/SM x 148 SMs x 1965 MHz (derived; 15.9/clk/SM measured)",
+                "hbm_frac": d["bytes"] / (d["ms"] * 1e-3) / 1e9 / hbm}
+        roof["traffic"] = ncu_traffic("kv_ssm_scan_kernel")
+    elif dom == "chunk_attn_fwd":
         ach = d["flops"] / (d["ms"] * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": ach, "peak": tf_burst, "unit": "TFLOP/s", "frac": ach / tf_burst,
                 "peak_source": f"{src} bf16 burst"}
@@ -353,8 +407,6 @@ def run_ours(args, ws, rank, local):
                 "peak_source": f"{src} HBM copy"}
         roof["traffic"] = ncu_traffic("kv_ssm_scan_kernel" if dom == "kv_ssm_scan" else "query_index_kernel")
     roof["kernel"] = dom
-    # the scan's binding unit is the exponential: also report it against 16 ex2/clk/SM at the max SM clock
-    exp_peak = 16 * 148 * 1.965e9
     scan = kernels["kv_ssm_scan"]
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
@@ -373,6 +425,8 @@ def run_ours(args, ws, rank, local):
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
     }
+    if ws == 1 and not args.no_decode:
+        out["decode"] = decode_bench(dev)
     if ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline()
     print(json.dumps(out), flush=True)
@@ -385,6 +439,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode-row measurement")
     ap.add_argument("--min-warmup-ms", type=float, default=500.0,
                     help="keep warming up at least this long so clocks have ramped (0 under a profiler)")
     args = ap.parse_args()

@@ -12,8 +12,7 @@
 // queries of one (sequence, head), longest key lists first.  An item's key
 // tiles (64 keys each) are first the chunk-end tiles 0..nbb(last query), then
 // the local band [ls(first query), last query]; both are plain TMA boxes.
-//   warp 4     TMA producer: Q (double buffered across items), then K/V tiles
-//              into a 3-stage ring
+//   warp 4     TMA producer: Q of each item, then K/V tiles into a 3-stage ring
 //   warp 5     one thread issues tcgen05.mma: S = Q K^T (M128 N64 K64) into
 //              TMEM, then O += P_j V_j (M128 N64 K64) into TMEM
 //   warps 0-3  softmax, one query row per thread: one tcgen05.ld round trip for
@@ -28,8 +27,9 @@
 // item's loads and QK^T overlap the current item's softmax and epilogue.
 // TMEM per CTA: S double buffer (2 x 64 columns) + O accumulators (2 x 64, by
 // item parity) = 256 columns, so two CTAs share an SM's 512; shared memory per
-// CTA: Q x 2, K/V x 3 stages, one P buffer (the next tile's softmax reaches its
-// P write only after the previous PV has finished).
+// CTA: Q x 1, K/V x 3 stages, P x 2 (a tile's softmax writes P while the PV of
+// the previous tile may still run).  The ring depth, Q buffers and CTAs per SM
+// are build-time settings; these values measured fastest on the bench workload.
 // Every wait is bounded; on a give-up the CTA raises ATTAMBA_DEV_TIMEOUT,
 // drains its own copies and MMAs, frees TMEM and leaves the tile unwritten.
 //
@@ -47,18 +47,28 @@ namespace {
 constexpr int kBM = 128;                                    // queries per work item (TMEM lanes)
 constexpr int kBN = 64;                                     // keys per tile
 constexpr int kDH = 64;
-constexpr int kStages = 3;
+#ifndef ATTAMBA_ATTN_STAGES
+#define ATTAMBA_ATTN_STAGES 3
+#endif
+#ifndef ATTAMBA_ATTN_QBUFS
+#define ATTAMBA_ATTN_QBUFS 1
+#endif
+#ifndef ATTAMBA_ATTN_CTAS_PER_SM
+#define ATTAMBA_ATTN_CTAS_PER_SM 2
+#endif
+constexpr int kStages = ATTAMBA_ATTN_STAGES;    // K/V ring depth
+constexpr int kQBufs = ATTAMBA_ATTN_QBUFS;      // Q buffers (2: the next item's Q loads during this item)
 constexpr int kThreads = 192;
-constexpr int kCtasPerSm = 2;
+constexpr int kCtasPerSm = ATTAMBA_ATTN_CTAS_PER_SM;
 constexpr int kMaxItems = 64;                               // work items per CTA (the host sizes the grid)
 constexpr uint32_t kQBytes = kBM * kDH * 2;                 // 16 KB: 128 rows x 128 bytes
 constexpr uint32_t kKVBytes = kBN * kDH * 2;                // 8 KB: 64 rows x 128 bytes
 constexpr uint32_t kPBytes = kBM * kBN * 2;                 // 16 KB: 128 rows x 64 keys bf16
-constexpr uint32_t kQOff = 0;                               // 2 Q buffers
-constexpr uint32_t kKOff = kQOff + 2 * kQBytes;             // kStages K tiles
+constexpr uint32_t kQOff = 0;                               // kQBufs Q buffers
+constexpr uint32_t kKOff = kQOff + kQBufs * kQBytes;        // kStages K tiles
 constexpr uint32_t kVOff = kKOff + kStages * kKVBytes;      // kStages V tiles
-constexpr uint32_t kPOff = kVOff + kStages * kKVBytes;      // 1 P buffer
-constexpr uint32_t kBarOff = kPOff + kPBytes;
+constexpr uint32_t kPOff = kVOff + kStages * kKVBytes;      // 2 P buffers
+constexpr uint32_t kBarOff = kPOff + 2 * kPBytes;
 constexpr uint32_t kItemOff = kBarOff + 256;
 constexpr uint32_t kSmemBytes = kItemOff + kMaxItems * 32 + 1024;   // + item table + alignment slack
 constexpr uint32_t kTmemCols = 256;
@@ -82,6 +92,8 @@ struct Bars {
   uint32_t tmem_base;
   int abort;
 };
+
+static_assert(sizeof(Bars) <= 256, "barrier block overflows its shared-memory slot");
 
 // One work item: 128 queries of one (sequence, head).  Items are numbered so
 // that the longest key lists (last query tiles) come first.
@@ -108,28 +120,6 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a, int item, int n_q
   it.NT = it.nbt + (band_len + kBN - 1) / kBN;
   it.chunk0 = a.bptr[it.b];
   return it;
-}
-
-// 128 consecutive 32-bit TMEM columns of this thread's lane, one wait
-__device__ __forceinline__ void tmem_ld128_sync(uint32_t taddr, uint32_t (&r)[128]) {
-#define ATT_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), "=r"(r[i + 5]), \
-                  "=r"(r[i + 6]), "=r"(r[i + 7])
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%128];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,"
-      "%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%129];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,"
-      "%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95}, [%130];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,"
-      "%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, "
-      "[%131];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : ATT_R8(0), ATT_R8(8), ATT_R8(16), ATT_R8(24), ATT_R8(32), ATT_R8(40), ATT_R8(48), ATT_R8(56),
-        ATT_R8(64), ATT_R8(72), ATT_R8(80), ATT_R8(88), ATT_R8(96), ATT_R8(104), ATT_R8(112), ATT_R8(120)
-      : "r"(taddr), "r"(taddr + 32), "r"(taddr + 64), "r"(taddr + 96)
-      : "memory");
-#undef ATT_R8
 }
 
 // 32 consecutive 32-bit columns from registers into this thread's TMEM lane, waited
@@ -224,8 +214,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const Item it = items[k];
         if (it.NT == 0) continue;
         const int64_t tok0 = (int64_t)it.b * n;
-        const int qb = wi & 1;
-        if (wi >= 2 && !mbar_wait_bounded(&bars->q_empty[qb], ((wi - 2) >> 1) & 1, abort_flag, kWaitNs)) {
+        const int qb = wi % kQBufs;
+        if (wi >= kQBufs && !mbar_wait_bounded(&bars->q_empty[qb], ((wi / kQBufs) - 1) & 1, abort_flag, kWaitNs)) {
           ok = false;
           break;
         }
@@ -253,7 +243,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       }
       if (!ok) *abort_flag = 1;
       // drain: the last copies into each buffer must land before the CTA may exit
-      for (int w = max(0, wi - 2); w < wi; ++w) mbar_wait_timeout(&bars->q_full[w & 1], (w >> 1) & 1, kWaitNs);
+      for (int w = max(0, wi - kQBufs); w < wi; ++w)
+        mbar_wait_timeout(&bars->q_full[w % kQBufs], (w / kQBufs) & 1, kWaitNs);
       for (int j = max(0, g - kStages); j < g; ++j)
         mbar_wait_timeout(&bars->kv_full[j % kStages], (j / kStages) & 1, kWaitNs);
     }
@@ -270,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             !mbar_wait_bounded(&bars->o_empty[ob], ((wi_of - 2) >> 1) & 1, abort_flag, kWaitNs))
           return false;
         tc_fence_after();
-        const uint32_t sp = smem_u32(smem + kPOff);
+        const uint32_t sp = smem_u32(smem + kPOff + sb * kPBytes);
         const uint32_t sv = smem_u32(smem + kVOff + st * kKVBytes);
 #pragma unroll
         for (int k = 0; k < kBN / 16; ++k) {
@@ -291,8 +282,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       for (int k = 0; ok && k < my_items; ++k) {
         const Item it = items[k];
         if (it.NT == 0) continue;
-        const int qb = wi & 1;
-        if (!mbar_wait_bounded(&bars->q_full[qb], (wi >> 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
+        const int qb = wi % kQBufs;
+        if (!mbar_wait_bounded(&bars->q_full[qb], (wi / kQBufs) & 1, abort_flag, kWaitNs)) { ok = false; break; }
         const uint32_t sq = smem_u32(smem + kQOff + qb * kQBytes);
         for (int j = 0; j < it.NT; ++j, ++g) {
           const int st = g % kStages, sb = g & 1;
@@ -323,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const int r = tid;  // query row within the tile == TMEM lane
     const float sl2 = a.scale * kLog2e;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    uint8_t* prow = smem + kPOff + r * 128;
+    uint8_t* prow0 = smem + kPOff + r * 128;
     const int sw = r & 7;
     int g = 0, wi = 0;
     bool ok = true;
@@ -406,10 +397,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
         // lazy rescale: keep the reference max unless the row max rose by more than 2^8
         const bool grow = (m_ref == -INFINITY) ? (mt > -INFINITY) : (mt > m_ref + kRescale);
-        // O and the P buffer are both free once the PV of the previous tile is done
-        if (g >= 1 && !wait_pv(g - 1)) { ok = false; break; }
         if (j > 0 && __any_sync(0xffffffffu, grow)) {
-          // O holds PV of the tiles before j: scale the rows that grow
+          // O holds PV of the tiles before j: once the last of them is done, scale the rows that grow
+          if (!wait_pv(g - 1)) { ok = false; break; }
           tc_fence_after();
           const float f = grow ? ex2(m_ref - mt) : 1.f;  // m_ref = -inf: O is still 0, f = 0
           uint32_t o0[32], o1[32];
@@ -428,6 +418,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
         const float2 sl2x2 = make_float2(sl2, sl2), negm = make_float2(-m_use, -m_use);
         float2 sum0 = make_float2(0.f, 0.f), sum1 = make_float2(0.f, 0.f);
+        // P buffer sb was last read by the PV of tile g - 2 (normally long finished)
+        if (g >= 2 && !wait_pv(g - 2)) { ok = false; break; }
+        uint8_t* prow = prow0 + sb * kPBytes;
 #pragma unroll
         for (int q = 0; q < kBN / 32; ++q) {
           // a 32-column chunk outside every lane's [lo, hi) needs no exponentials

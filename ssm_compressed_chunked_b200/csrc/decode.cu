@@ -69,14 +69,18 @@ __global__ void __launch_bounds__(128) decode_ssm_kernel(DecodeArgs a) {
   const float dx = delta * __bfloat162float(x[(size_t)b * D + d]);
   float* st = c.state + ((size_t)(s * c.B + b) * kNS) * D + d;
   const float* A = a.A[s] + (size_t)d * kNS;
+  // all 16 state loads are issued before any use (one memory latency, not sixteen)
+  float h[kNS];
+#pragma unroll
+  for (int n = 0; n < kNS; ++n) h[n] = start ? 0.f : st[(size_t)n * D];
   float y = 0.f;
 #pragma unroll
   for (int n = 0; n < kNS; ++n) {
-    float h = start ? 0.f : st[(size_t)n * D];
-    h = fmaf(ex2(delta * A[n] * kLog2e), h, dx * __bfloat162float(Bm[n]));
-    st[(size_t)n * D] = h;
-    y = fmaf(__bfloat162float(Cm[n]), h, y);
+    h[n] = fmaf(ex2(delta * A[n] * kLog2e), h[n], dx * __bfloat162float(Bm[n]));
+    y = fmaf(__bfloat162float(Cm[n]), h[n], y);
   }
+#pragma unroll
+  for (int n = 0; n < kNS; ++n) st[(size_t)n * D] = h[n];
   const int head = d / c.dh, e = d - head * c.dh;
   const __nv_bfloat16 yb = __float2bfloat16_rn(y);
   __nv_bfloat16* ring = static_cast<__nv_bfloat16*>(s == 0 ? c.Kr : c.Vr);
@@ -144,8 +148,9 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(DecodeArgs a)
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 
-  for (int kk = kb + warp * 4; kk < ke; kk += 16 * kUnroll) {
-    uint4 kr[kUnroll], vr[kUnroll];
+  // Keys are processed in sweeps of 16 (4 warps x 4 key groups) x kUnroll; two register
+  // buffers alternate so one sweep's loads are in flight while the other is computed.
+  auto load_sweep = [&](int kk, uint4 (&kr)[kUnroll], uint4 (&vr)[kUnroll]) {
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int k = kk + u * 16 + g;
@@ -166,6 +171,8 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(DecodeArgs a)
         vr[u] = make_uint4(0, 0, 0, 0);
       }
     }
+  };
+  auto compute_sweep = [&](int kk, const uint4 (&kr)[kUnroll], const uint4 (&vr)[kUnroll]) {
     float sc[kUnroll];
     float mt = -INFINITY;
 #pragma unroll
@@ -198,6 +205,22 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(DecodeArgs a)
       }
       m = m_new;
     }
+  };
+  constexpr int kSweep = 16 * kUnroll;
+  uint4 kA[kUnroll], vA[kUnroll], kB[kUnroll], vB[kUnroll];
+  int kk = kb + warp * 4;
+  if (kk < ke) load_sweep(kk, kA, vA);
+  while (kk < ke) {
+    const bool more = kk + kSweep < ke;
+    if (more) load_sweep(kk + kSweep, kB, vB);
+    compute_sweep(kk, kA, vA);
+    if (!more) break;
+    kk += kSweep;
+    const bool more2 = kk + kSweep < ke;
+    if (more2) load_sweep(kk + kSweep, kA, vA);
+    compute_sweep(kk, kB, vB);
+    if (!more2) break;
+    kk += kSweep;
   }
 
   // merge the four key groups of the warp (lanes with the same slice: xor 8, 16)

@@ -38,15 +38,18 @@
 #define ATTAMBA_SCAN_CPT 2
 #endif
 #ifndef ATTAMBA_SCAN_MINB
-#define ATTAMBA_SCAN_MINB 4
+#define ATTAMBA_SCAN_MINB 3
 #endif
 
 namespace attamba {
 
 namespace {
 constexpr int kScanThreads = 128;
-constexpr int kStageTokens = 64;
-constexpr int kMaxChunksPerBlock = 64;
+#ifndef ATTAMBA_SCAN_TOKENS
+#define ATTAMBA_SCAN_TOKENS 128
+#endif
+constexpr int kStageTokens = 64;       // B/C staging window (even, so token pairs never straddle one)
+constexpr int kMaxChunksPerBlock = 256;
 constexpr int kNS = 16;
 constexpr int kNP = kNS / 2;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -125,30 +128,6 @@ template <> struct Vec<__nv_bfloat16, 2> {
   }
   static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[2]) {
     *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v[0], v[1]);
-  }
-};
-template <> struct Vec<__nv_bfloat16, 4> {
-  using raw = uint2;
-  static __device__ __forceinline__ raw load(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint2*>(p)); }
-  static __device__ __forceinline__ void unpack(raw r, float (&v)[4]) {
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
-    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
-  }
-  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[4]) {
-    __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
-    uint2 r;
-    r.x = *reinterpret_cast<uint32_t*>(&a);
-    r.y = *reinterpret_cast<uint32_t*>(&b);
-    *reinterpret_cast<uint2*>(p) = r;
-  }
-};
-template <> struct Vec<float, 4> {
-  using raw = float4;
-  static __device__ __forceinline__ raw load(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
-  static __device__ __forceinline__ void unpack(raw r, float (&v)[4]) { v[0] = r.x; v[1] = r.y; v[2] = r.z; v[3] = r.w; }
-  static __device__ __forceinline__ void store(float* p, const float (&v)[4]) {
-    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
   }
 };
 template <> struct Vec<float, 2> {
@@ -246,30 +225,33 @@ __global__ void __launch_bounds__(kScanThreads, ATTAMBA_SCAN_MINB) kv_ssm_scan_k
   int ci = 0;                 // chunk of the current token, relative to c_begin
   int next_start = sCu[1];
 
-  // delta of the next token, computed one token ahead from loads issued one token ahead
-  float dl_n[CPT], dx_n[CPT];
-  auto delta_of = [&](typename V::raw xr, typename V::raw zr) {
+  // Software pipeline over token pairs: the deltas of the pair being computed
+  // come from loads issued one pair earlier, and the loads for the pair after
+  // next are issued once the registers they land in have been consumed.
+  float dlA[CPT], dxA[CPT], dlB[CPT], dxB[CPT];
+  typename V::raw xA, zA, xB, zB;
+  auto delta_of = [&](typename V::raw xr, typename V::raw zr, float (&dl)[CPT], float (&dx)[CPT]) {
     float xv[CPT], zv[CPT];
     V::unpack(xr, xv);
     V::unpack(zr, zv);
 #pragma unroll
     for (int cc = 0; cc < CPT; ++cc) {
-      dl_n[cc] = softplus_f(zv[cc] + st.bias[cc]);
-      dx_n[cc] = dl_n[cc] * xv[cc];
+      dl[cc] = softplus_f(zv[cc] + st.bias[cc]);
+      dx[cc] = dl[cc] * xv[cc];
     }
   };
-  if (active) delta_of(V::load(x + t_begin * D), V::load(dt + t_begin * D));
+  auto tok = [&](int t) { return min(t, t_end - 1); };  // clamped: harmless reloads past the end
+  if (active) {
+    delta_of(V::load(x + tok(t_begin) * D), V::load(dt + tok(t_begin) * D), dlA, dxA);
+    delta_of(V::load(x + tok(t_begin + 1) * D), V::load(dt + tok(t_begin + 1) * D), dlB, dxB);
+    xA = V::load(x + tok(t_begin + 2) * D); zA = V::load(dt + tok(t_begin + 2) * D);
+    xB = V::load(x + tok(t_begin + 3) * D); zB = V::load(dt + tok(t_begin + 3) * D);
+  }
 
-  auto step = [&](int t, const float* bc) {
-    const int tn = min(t + 1, t_end - 1);  // the next token (clamped: a harmless reload at the end)
-    const typename V::raw xr = V::load(x + tn * D), zr = V::load(dt + tn * D);
-    float dl[CPT], dx[CPT], dmax = 0.f;
+  auto step = [&](int t, const float* bc, const float (&dl)[CPT], const float (&dx)[CPT]) {
+    float dmax = 0.f;
 #pragma unroll
-    for (int cc = 0; cc < CPT; ++cc) {
-      dl[cc] = dl_n[cc];
-      dx[cc] = dx_n[cc];
-      dmax = fmaxf(dmax, dl[cc]);
-    }
+    for (int cc = 0; cc < CPT; ++cc) dmax = fmaxf(dmax, dl[cc]);
     const bool reset = (t == next_start);
     ci += reset ? 1 : 0;
     next_start = sCu[ci + 1];
@@ -279,7 +261,6 @@ __global__ void __launch_bounds__(kScanThreads, ATTAMBA_SCAN_MINB) kv_ssm_scan_k
     scan_token<T, CPT, POLY_PAIRS>(st, bc, dl, dx, reset, poly_ok, y);
     V::store(out + t * D, y);
     if (outc != nullptr && t + 1 == next_start) V::store(outc + (c_begin + ci) * D + d0, y);
-    delta_of(xr, zr);
   };
 
   for (int tb = t_begin; tb < t_end; tb += kStageTokens) {
@@ -292,20 +273,24 @@ __global__ void __launch_bounds__(kScanThreads, ATTAMBA_SCAN_MINB) kv_ssm_scan_k
     }
     __syncthreads();
     if (!active) continue;
-    int k = 0;
-    for (; k + 1 < nt; k += 2) {  // two tokens per iteration: their independent work interleaves
-      step(tb + k, &sBC[k][0]);
-      step(tb + k + 1, &sBC[k + 1][0]);
+    // token pairs are counted from t_begin, so the pipeline stays aligned across windows
+    for (int k = 0; k < nt; k += 2) {
+      const int t = tb + k;
+      step(t, &sBC[k][0], dlA, dxA);
+      if (k + 1 < nt) step(t + 1, &sBC[k + 1][0], dlB, dxB);
+      delta_of(xA, zA, dlA, dxA);
+      delta_of(xB, zB, dlB, dxB);
+      xA = V::load(x + tok(t + 4) * D); zA = V::load(dt + tok(t + 4) * D);
+      xB = V::load(x + tok(t + 5) * D); zB = V::load(dt + tok(t + 5) * D);
     }
-    if (k < nt) step(tb + k, &sBC[k][0]);
   }
 }
 }  // namespace
 
 cudaError_t launch_kv_ssm_scan(attamba_dtype_t dtype, const ScanArgs& a, cudaStream_t s) {
   constexpr int CPT = ATTAMBA_SCAN_CPT;
-  // about 64 tokens of chunks per block
-  int64_t cpb = (64 * (int64_t)a.n_chunks) / (a.T > 0 ? a.T : 1);
+  // about ATTAMBA_SCAN_TOKENS tokens of chunks per block
+  int64_t cpb = ((int64_t)ATTAMBA_SCAN_TOKENS * a.n_chunks) / (a.T > 0 ? a.T : 1);
   if (cpb < 1) cpb = 1;
   if (cpb > kMaxChunksPerBlock) cpb = kMaxChunksPerBlock;
   if ((a.n_chunks + cpb - 1) / cpb > 65535) return cudaErrorInvalidValue;
