@@ -12,26 +12,33 @@
 // queries of one (sequence, head), longest key lists first.  An item's key
 // tiles (64 keys each) are first the chunk-end tiles 0..nbb(last query), then
 // the local band [ls(first query), last query]; both are plain TMA boxes.
-//   warp 4     TMA producer: Q of each item, then K/V tiles into a 3-stage ring
-//   warp 5     one thread issues tcgen05.mma: S = Q K^T (M128 N64 K64) into
-//              TMEM, then O += P_j V_j (M128 N64 K64) into TMEM
-//   warps 0-3  softmax, one query row per thread: one tcgen05.ld round trip for
-//              its S row, masking only where a row's key range cuts the tile,
-//              32-column chunks outside every row's range skipped, online
-//              max/sum in fp32, P as bf16 into shared memory (the A operand of
-//              the PV MMA)
-// O accumulates in TMEM across an item's tiles.  P uses a reference max that
-// is raised (and O, l rescaled in TMEM) only when a row's max grows by more
-// than 2^8, so P <= 2^8 and the rescale is rare; the final O / l is exact
-// whatever reference was used.  Tile counters run across items, so the next
-// item's loads and QK^T overlap the current item's softmax and epilogue.
-// TMEM per CTA: S double buffer (2 x 64 columns) + O accumulators (2 x 64, by
-// item parity) = 256 columns, so two CTAs share an SM's 512; shared memory per
-// CTA: Q x 1, K/V x 3 stages, P x 2 (a tile's softmax writes P while the PV of
-// the previous tile may still run).  The ring depth, Q buffers and CTAs per SM
-// are build-time settings; these values measured fastest on the bench workload.
-// Every wait is bounded; on a give-up the CTA raises ATTAMBA_DEV_TIMEOUT,
-// drains its own copies and MMAs, frees TMEM and leaves the tile unwritten.
+//   warp 4     TMA producer: Q of each item (two buffers), then K/V tiles into
+//              a 3-stage ring
+//   warp 5     one thread issues tcgen05.mma: S = Q K^T (M128 N64 K64, both
+//              operands in shared memory) into TMEM, then O += P V (M128 N64
+//              K64, P read from TMEM, V from shared memory)
+//   warps 0-3  softmax, one query row per thread: one tcgen05.ld for its S row,
+//              masking only where the row's key range cuts the tile, 32-column
+//              chunks outside every row's range skipped, online max/sum in
+//              fp32, P as bf16 pairs back into TMEM with one tcgen05.st
+// TMEM per CTA (256 columns): S in two buffers of 64, P in two of 32, O 64.
+// With S and P double-buffered the QK of tile g + 1 and the PV of tile g - 1
+// run while the softmax works on tile g; the softmax waits only for the PV
+// that last read the P buffer it is about to fill (tile g - 2).  Because the
+// four softmax warps can then drift up to two tiles apart, every barrier they
+// arrive on exists per buffer.  O accumulates in TMEM across an item's tiles;
+// P uses a reference max that is raised (and O, l rescaled in TMEM) only when
+// a row's max grows by more than 2^8, so P <= 2^8 and the rescale is rare; the
+// final O / l is exact whatever reference was used.  A full 128-row tile of O
+// leaves through a shared-memory staging tile and one TMA store; a partial
+// tile (the end of a sequence) is written row by row.
+//
+// Measured limits (B200, bench workload): the exponentials of a 64-column
+// tile cost 512 cycles of the multi-function unit per warp, so two CTAs per SM
+// keep it about 60% busy; the rest of a tile's time is barrier and TMEM
+// latency.  A third CTA does not fit (TMEM, shared memory); eight softmax
+// warps with the 16-lane TMEM shapes, 128-key tiles, and moving a share of the
+// exponentials to an FMA-pipe polynomial all measured slower.
 //
 // f32 kernel: one thread per (query, head) on the CUDA cores, same key sets,
 // fp32 online softmax (the fp32 tensor-core kinds round to tf32).
@@ -50,49 +57,52 @@ constexpr int kDH = 64;
 #ifndef ATTAMBA_ATTN_STAGES
 #define ATTAMBA_ATTN_STAGES 3
 #endif
-#ifndef ATTAMBA_ATTN_QBUFS
-#define ATTAMBA_ATTN_QBUFS 1
-#endif
 #ifndef ATTAMBA_ATTN_CTAS_PER_SM
 #define ATTAMBA_ATTN_CTAS_PER_SM 2
 #endif
-constexpr int kStages = ATTAMBA_ATTN_STAGES;    // K/V ring depth
-constexpr int kQBufs = ATTAMBA_ATTN_QBUFS;      // Q buffers (2: the next item's Q loads during this item)
+constexpr int kStages = ATTAMBA_ATTN_STAGES;                // K/V ring depth
 constexpr int kThreads = 192;
 constexpr int kCtasPerSm = ATTAMBA_ATTN_CTAS_PER_SM;
 constexpr int kMaxItems = 64;                               // work items per CTA (the host sizes the grid)
 constexpr uint32_t kQBytes = kBM * kDH * 2;                 // 16 KB: 128 rows x 128 bytes
 constexpr uint32_t kKVBytes = kBN * kDH * 2;                // 8 KB: 64 rows x 128 bytes
-constexpr uint32_t kPBytes = kBM * kBN * 2;                 // 16 KB: 128 rows x 64 keys bf16
-constexpr uint32_t kQOff = 0;                               // kQBufs Q buffers
-constexpr uint32_t kKOff = kQOff + kQBufs * kQBytes;        // kStages K tiles
+constexpr uint32_t kQOff = 0;                               // two Q tiles
+constexpr uint32_t kKOff = kQOff + 2 * kQBytes;             // kStages K tiles
 constexpr uint32_t kVOff = kKOff + kStages * kKVBytes;      // kStages V tiles
-constexpr uint32_t kPOff = kVOff + kStages * kKVBytes;      // 2 P buffers
-constexpr uint32_t kBarOff = kPOff + 2 * kPBytes;
+constexpr uint32_t kOOff = kVOff + kStages * kKVBytes;      // O staging tile for the TMA store
+constexpr uint32_t kBarOff = kOOff + kQBytes;
 constexpr uint32_t kItemOff = kBarOff + 256;
 constexpr uint32_t kSmemBytes = kItemOff + kMaxItems * 32 + 1024;   // + item table + alignment slack
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kSCol = 0;     // S buffers at columns 0 and 64
-constexpr uint32_t kOCol = 128;   // O accumulators at columns 128 and 192 (by item parity)
+constexpr uint32_t kTmemCols = 256;                         // power of two, >= 32
+constexpr uint32_t kSCol = 0;                               // S, two buffers: columns 0..63, 64..127 (fp32)
+constexpr uint32_t kPCol = 2 * kBN;                         // P, two buffers: columns 128..159, 160..191 (bf16 pairs)
+constexpr uint32_t kOCol = 3 * kBN;                         // O: columns 192..255 (fp32)
 constexpr uint64_t kWaitNs = 4000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.f;   // O is rescaled only when a row's max grows by more than 2^8
+static_assert(kOCol + kDH <= kTmemCols, "TMEM columns");
 
+// Double-buffered resources (Q, S, P) use barrier pairs: use u of the resource is
+// buffer u & 1, phase u >> 1 of that buffer's barrier; the K/V ring completes once
+// per use of a stage.  The softmax warps may drift up to two key tiles apart, so
+// every barrier they arrive on is per buffer: an arrival for tile g + 1 must not
+// count towards tile g.
 struct Bars {
   uint64_t q_full[2];
   uint64_t q_empty[2];
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t pv_done[2];   // PV of global tile g completes phase g/2 of pv_done[g & 1]
-  uint64_t o_empty[2];   // the epilogue has read O accumulator [item parity]
+  uint64_t s_full[2];    // QK of tile g done (tcgen05.commit)
+  uint64_t s_empty[2];   // every softmax thread has read S of tile g (128 arrivals)
+  uint64_t p_full[2];    // every softmax thread has written P of tile g (128 arrivals)
+  uint64_t pv_done[2];   // PV of tile g done (tcgen05.commit)
   uint64_t mma_done;
+  uint64_t o_ready;      // every softmax thread has written its row of the O staging tile (128 arrivals)
+  uint64_t o_free;       // the last TMA store has finished reading the staging tile
   uint32_t tmem_base;
   int abort;
 };
-
 static_assert(sizeof(Bars) <= 256, "barrier block overflows its shared-memory slot");
 
 // One work item: 128 queries of one (sequence, head).  Items are numbered so
@@ -122,19 +132,40 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a, int item, int n_q
   return it;
 }
 
-// 32 consecutive 32-bit columns from registers into this thread's TMEM lane, waited
-__device__ __forceinline__ void tmem_st32_sync(uint32_t taddr, const uint32_t (&r)[32]) {
+// 64 consecutive 32-bit TMEM columns of this thread's lane, one wait
+__device__ __forceinline__ void tmem_ld64_sync(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr)
+      : "memory");
+}
+
+// 32 consecutive 32-bit columns from registers into this thread's TMEM lane (not waited)
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n\t"
-      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
       "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
@@ -157,10 +188,25 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return d;
 }
 
+// 3-D tiled tensor store from this CTA's shared memory (bulk async group)
+__device__ __forceinline__ void tma_store_3d(const void* tmap, const void* src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(tmap),
+               "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// the previous stores have finished reading shared memory
+__device__ __forceinline__ void tma_store_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// the previous stores are complete
+__device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     chunk_attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc,
-                           const __grid_constant__ CUtensorMap tm_vc, AttnArgs a) {
+                           const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_o,
+                           AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);
@@ -180,16 +226,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   }
   for (int k = tid; k < my_items; k += kThreads) items[k] = decode_item(a, blockIdx.x + k * gridDim.x, n_qt);
   if (warp == 4 && lane == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->q_full[i], 1);
-      mbar_init(&bars->q_empty[i], 1);
-      mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], kBM);
-      mbar_init(&bars->pv_done[i], 1);
-      mbar_init(&bars->o_empty[i], kBM);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->q_full[b], 1);
+      mbar_init(&bars->q_empty[b], 1);
+      mbar_init(&bars->s_full[b], 1);
+      mbar_init(&bars->s_empty[b], kBM);
+      mbar_init(&bars->pv_done[b], 1);
+      mbar_init(&bars->p_full[b], kBM);
     }
     for (int i = 0; i < kStages; ++i) { mbar_init(&bars->kv_full[i], 1); mbar_init(&bars->kv_empty[i], 1); }
     mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->o_ready, kBM);
+    mbar_init(&bars->o_free, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -207,15 +255,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_kc); tma_prefetch_desc(&tm_vc);
+      tma_prefetch_desc(&tm_kc); tma_prefetch_desc(&tm_vc); tma_prefetch_desc(&tm_o);
       int g = 0, wi = 0;
       bool ok = true;
       for (int k = 0; ok && k < my_items; ++k) {
         const Item it = items[k];
         if (it.NT == 0) continue;
         const int64_t tok0 = (int64_t)it.b * n;
-        const int qb = wi % kQBufs;
-        if (wi >= kQBufs && !mbar_wait_bounded(&bars->q_empty[qb], ((wi / kQBufs) - 1) & 1, abort_flag, kWaitNs)) {
+        const int qb = wi & 1;
+        if (wi >= 2 && !mbar_wait_bounded(&bars->q_empty[qb], ((wi - 2) >> 1) & 1, abort_flag, kWaitNs)) {
           ok = false;
           break;
         }
@@ -230,21 +278,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             break;
           }
           mbar_arrive_expect_tx(&bars->kv_full[st], 2 * kKVBytes);
-          if (j < it.nbt) {
-            const int row = it.chunk0 + j * kBN;
-            tma_load_3d(smem + kKOff + st * kKVBytes, &tm_kc, 0, it.h, row, &bars->kv_full[st]);
-            tma_load_3d(smem + kVOff + st * kKVBytes, &tm_vc, 0, it.h, row, &bars->kv_full[st]);
-          } else {
-            const int row = (int)(tok0 + it.ls_first + (j - it.nbt) * kBN);
-            tma_load_3d(smem + kKOff + st * kKVBytes, &tm_k, 0, it.h, row, &bars->kv_full[st]);
-            tma_load_3d(smem + kVOff + st * kKVBytes, &tm_v, 0, it.h, row, &bars->kv_full[st]);
-          }
+          const bool bnd = j < it.nbt;
+          const int row = bnd ? it.chunk0 + j * kBN : (int)(tok0 + it.ls_first + (j - it.nbt) * kBN);
+          tma_load_3d(smem + kKOff + st * kKVBytes, bnd ? &tm_kc : &tm_k, 0, it.h, row, &bars->kv_full[st]);
+          tma_load_3d(smem + kVOff + st * kKVBytes, bnd ? &tm_vc : &tm_v, 0, it.h, row, &bars->kv_full[st]);
         }
       }
       if (!ok) *abort_flag = 1;
       // drain: the last copies into each buffer must land before the CTA may exit
-      for (int w = max(0, wi - kQBufs); w < wi; ++w)
-        mbar_wait_timeout(&bars->q_full[w % kQBufs], (w / kQBufs) & 1, kWaitNs);
+      for (int u = max(0, wi - 2); u < wi; ++u) mbar_wait_timeout(&bars->q_full[u & 1], (u >> 1) & 1, kWaitNs);
       for (int j = max(0, g - kStages); j < g; ++j)
         mbar_wait_timeout(&bars->kv_full[j % kStages], (j / kStages) & 1, kWaitNs);
     }
@@ -253,58 +295,52 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (lane == 0) {
       const uint32_t idesc_qk = umma_idesc_bf16(kBM, kBN, 0, 0);
       const uint32_t idesc_pv = umma_idesc_bf16(kBM, kDH, 0, 1);
-      // PV of tile gg into the O accumulator of item wi_of (first tile of the item overwrites)
-      auto issue_pv = [&](int gg, int wi_of, bool first) -> bool {
-        const int sb = gg & 1, st = gg % kStages, ob = wi_of & 1;
-        if (!mbar_wait_bounded(&bars->p_full[sb], (gg >> 1) & 1, abort_flag, kWaitNs)) return false;
-        if (first && wi_of >= 2 &&
-            !mbar_wait_bounded(&bars->o_empty[ob], ((wi_of - 2) >> 1) & 1, abort_flag, kWaitNs))
-          return false;
+      // PV of tile gg: O (+)= P V with P from TMEM buffer gg & 1 (8 columns per 16 keys) and V
+      // from shared memory (MN-major, 2048 bytes per 16 keys); the first tile of an item overwrites O
+      auto issue_pv = [&](int gg, bool first) -> bool {
+        const int st = gg % kStages;
+        if (!mbar_wait_bounded(&bars->p_full[gg & 1], (gg >> 1) & 1, abort_flag, kWaitNs)) return false;
         tc_fence_after();
-        const uint32_t sp = smem_u32(smem + kPOff + sb * kPBytes);
         const uint32_t sv = smem_u32(smem + kVOff + st * kKVBytes);
 #pragma unroll
-        for (int k = 0; k < kBN / 16; ++k) {
-          // A = P (K-major: 128 rows x 64 keys, 32 bytes per 16 keys)
-          const uint64_t adesc = umma_desc_sw128(sp + k * 32, 16, 1024);
-          // B = V (MN-major: 16 keys = two 8-row groups of 1024 bytes)
-          const uint64_t bdesc = umma_desc_sw128(sv + k * 2048, 16, 1024);
-          umma_bf16(tmem + kOCol + ob * kDH, adesc, bdesc, idesc_pv, (first && k == 0) ? 0u : 1u);
-        }
-        umma_commit(&bars->pv_done[sb]);
+        for (int k = 0; k < kBN / 16; ++k)
+          umma_bf16_ts(tmem + kOCol, tmem + kPCol + (gg & 1) * (kBN / 2) + k * 8,
+                       umma_desc_sw128(sv + k * 2048, 16, 1024), idesc_pv, (first && k == 0) ? 0u : 1u);
+        umma_commit(&bars->pv_done[gg & 1]);
         umma_commit(&bars->kv_empty[st]);
         return true;
       };
       int g = 0, wi = 0;
-      int pend_wi = 0;
       bool pend_first = false;
       bool ok = true;
       for (int k = 0; ok && k < my_items; ++k) {
         const Item it = items[k];
         if (it.NT == 0) continue;
-        const int qb = wi % kQBufs;
-        if (!mbar_wait_bounded(&bars->q_full[qb], (wi / kQBufs) & 1, abort_flag, kWaitNs)) { ok = false; break; }
+        const int qb = wi & 1;
+        if (!mbar_wait_bounded(&bars->q_full[qb], (wi >> 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
         const uint32_t sq = smem_u32(smem + kQOff + qb * kQBytes);
         for (int j = 0; j < it.NT; ++j, ++g) {
-          const int st = g % kStages, sb = g & 1;
+          const int st = g % kStages;
           if (!mbar_wait_bounded(&bars->kv_full[st], (g / kStages) & 1, abort_flag, kWaitNs)) { ok = false; break; }
+          // S buffer g & 1 was last read by the softmax for tile g - 2
+          if (g >= 2 && !mbar_wait_bounded(&bars->s_empty[g & 1], ((g - 2) >> 1) & 1, abort_flag, kWaitNs)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t sk = smem_u32(smem + kKOff + st * kKVBytes);
 #pragma unroll
-          for (int kk = 0; kk < kDH / 16; ++kk) {
-            const uint64_t adesc = umma_desc_sw128(sq + kk * 32, 16, 1024);
-            const uint64_t bdesc = umma_desc_sw128(sk + kk * 32, 16, 1024);
-            umma_bf16(tmem + kSCol + sb * kBN, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&bars->s_full[sb]);
-          if (j == it.NT - 1) umma_commit(&bars->q_empty[qb]);  // Q buffer free once its last QK is done
-          if (g >= 1 && !issue_pv(g - 1, pend_wi, pend_first)) { ok = false; break; }
-          pend_wi = wi;
+          for (int kk = 0; kk < kDH / 16; ++kk)
+            umma_bf16(tmem + kSCol + (g & 1) * kBN, umma_desc_sw128(sq + kk * 32, 16, 1024),
+                      umma_desc_sw128(sk + kk * 32, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          umma_commit(&bars->s_full[g & 1]);
+          if (j == it.NT - 1) umma_commit(&bars->q_empty[qb]);  // Q free once the item's last QK is done
+          if (g >= 1 && !issue_pv(g - 1, pend_first)) { ok = false; break; }
           pend_first = (j == 0);
         }
         ++wi;
       }
-      if (ok && g >= 1) ok = issue_pv(g - 1, pend_wi, pend_first);
+      if (ok && g >= 1) ok = issue_pv(g - 1, pend_first);
       if (!ok) *abort_flag = 1;
       umma_commit(&bars->mma_done);  // every MMA issued above has finished when this arrives
       mbar_wait_timeout(&bars->mma_done, 0, kWaitNs);
@@ -314,34 +350,26 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const int r = tid;  // query row within the tile == TMEM lane
     const float sl2 = a.scale * kLog2e;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    uint8_t* prow0 = smem + kPOff + r * 128;
+    const uint32_t o_tmem = lane_base + kOCol;
+    uint8_t* orow = smem + kOOff + r * 128;   // this row of the O staging tile
     const int sw = r & 7;
-    int g = 0, wi = 0;
+    int g = 0;
     bool ok = true;
-    // wait for the PV of global tile gg (consecutive waits per P buffer; verdict warp-uniform)
+    int n_stores = 0;   // TMA stores of the staging tile issued so far (phases of o_ready / o_free)
+    // wait for the PV of tile gg (barrier gg & 1, its phase gg >> 1; verdict warp-uniform)
     auto wait_pv = [&](int gg) -> bool {
-      return __all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done[gg & 1], (gg >> 1) & 1, abort_flag, kWaitNs));
+      return __all_sync(0xffffffffu,
+                        mbar_wait_bounded(&bars->pv_done[gg & 1], (gg >> 1) & 1, abort_flag, kWaitNs));
     };
-    // this row's key range of the first item, then prefetched one item ahead
-    int nx_ls = 0, nx_nbb = 0;
-    if (my_items > 0 && items[0].q0 + r <= items[0].q_last) {
-      const int64_t tok = (int64_t)items[0].b * n + items[0].q0 + r;
-      nx_ls = a.ls[tok];
-      nx_nbb = a.nbb[tok];
-    }
     for (int k = 0; ok && k < my_items; ++k) {
       const Item it = items[k];
       const int64_t tok0 = (int64_t)it.b * n;
       const int i = it.q0 + r;
       const bool row_ok = i <= it.q_last;
-      const int my_ls = nx_ls, my_nbb = nx_nbb;
-      if (k + 1 < my_items) {
-        const Item nx = items[k + 1];
-        if (nx.q0 + r <= nx.q_last) {
-          const int64_t tok = (int64_t)nx.b * n + nx.q0 + r;
-          nx_ls = a.ls[tok];
-          nx_nbb = a.nbb[tok];
-        }
+      int my_ls = 0, my_nbb = 0;
+      if (row_ok) {
+        my_ls = a.ls[tok0 + i];
+        my_nbb = a.nbb[tok0 + i];
       }
       if (it.NT == 0) {  // every row of the item has an empty key set
         if (row_ok) {
@@ -352,11 +380,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         }
         continue;
       }
-      const int ob = wi & 1;
-      const uint32_t o_tmem = lane_base + kOCol + ob * kDH;
       float m_ref = -INFINITY, l_run = 0.f;  // P of this item is exp2(s * sl2 - m_ref)
       for (int j = 0; j < it.NT; ++j, ++g) {
-        const int sb = g & 1;
         int lo, hi;
         if (j < it.nbt) {
           lo = 0;
@@ -367,130 +392,156 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           hi = min(max(i - j0 + 1, 0), kBN);
         }
         if (!row_ok) { lo = 0; hi = 0; }
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[sb], (g >> 1) & 1, abort_flag, kWaitNs))) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[g & 1], (g >> 1) & 1, abort_flag, kWaitNs))) {
           ok = false;
           break;
         }
         tc_fence_after();
         uint32_t sr[kBN];
-        tmem_ld32_sync(lane_base + kSCol + sb * kBN, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32_sync(lane_base + kSCol + sb * kBN + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        float s[kBN];
-        // row max of the raw scores over the valid columns [lo, hi)
-        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-        if (lo == 0 && hi == kBN) {
-#pragma unroll
-          for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c]);
-        } else {
+        tmem_ld64_sync(lane_base + kSCol + (g & 1) * kBN, &sr[0]);
+        tc_fence_before();
+        mbar_arrive(&bars->s_empty[g & 1]);
+        // row max of the raw scores over the valid columns [lo, hi); masked columns become -inf in place
+        if (lo != 0 || hi != kBN) {
           const unsigned span = (unsigned)(hi - lo);
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
-            s[c] = ((unsigned)(c - lo) < span) ? __uint_as_float(sr[c]) : -INFINITY;
+            if ((unsigned)(c - lo) >= span) sr[c] = 0xff800000u;
         }
+#define S_(c) __uint_as_float(sr[c])
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
         for (int c = 0; c < kBN; c += 8) {
-          mx0 = max3(mx0, s[c], s[c + 1]);
-          mx1 = max3(mx1, s[c + 2], s[c + 3]);
-          mx2 = max3(mx2, s[c + 4], s[c + 5]);
-          mx3 = max3(mx3, s[c + 6], s[c + 7]);
+          mx0 = max3(mx0, S_(c), S_(c + 1));
+          mx1 = max3(mx1, S_(c + 2), S_(c + 3));
+          mx2 = max3(mx2, S_(c + 4), S_(c + 5));
+          mx3 = max3(mx3, S_(c + 6), S_(c + 7));
         }
         const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
         // lazy rescale: keep the reference max unless the row max rose by more than 2^8
         const bool grow = (m_ref == -INFINITY) ? (mt > -INFINITY) : (mt > m_ref + kRescale);
-        if (j > 0 && __any_sync(0xffffffffu, grow)) {
-          // O holds PV of the tiles before j: once the last of them is done, scale the rows that grow
-          if (!wait_pv(g - 1)) { ok = false; break; }
-          tc_fence_after();
-          const float f = grow ? ex2(m_ref - mt) : 1.f;  // m_ref = -inf: O is still 0, f = 0
-          uint32_t o0[32], o1[32];
-          tmem_ld32_sync(o_tmem, o0);
-          tmem_ld32_sync(o_tmem + 32, o1);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            o0[c] = __float_as_uint(__uint_as_float(o0[c]) * f);
-            o1[c] = __float_as_uint(__uint_as_float(o1[c]) * f);
-          }
-          tmem_st32_sync(o_tmem, o0);
-          tmem_st32_sync(o_tmem + 32, o1);
-          l_run *= f;
+        const bool rescale = j > 0 && __any_sync(0xffffffffu, grow);
+        // factor that brings this row's O and l from the old reference to the new one
+        // (m_ref = -inf: O and l are still 0, the factor is 0)
+        const float fscale = (grow && j > 0) ? ex2(m_ref - mt) : 1.f;
+        if (grow) {
+          l_run *= fscale;
+          m_ref = mt;
         }
-        if (grow) m_ref = mt;
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
         const float2 sl2x2 = make_float2(sl2, sl2), negm = make_float2(-m_use, -m_use);
         float2 sum0 = make_float2(0.f, 0.f), sum1 = make_float2(0.f, 0.f);
-        // P buffer sb was last read by the PV of tile g - 2 (normally long finished)
-        if (g >= 2 && !wait_pv(g - 2)) { ok = false; break; }
-        uint8_t* prow = prow0 + sb * kPBytes;
+        uint32_t pk[kBN / 2];
 #pragma unroll
         for (int q = 0; q < kBN / 32; ++q) {
           // a 32-column chunk outside every lane's [lo, hi) needs no exponentials
           const bool need = __any_sync(0xffffffffu, lo < q * 32 + 32 && hi > q * 32);
-          uint32_t pk[16];
           if (need) {
 #pragma unroll
             for (int c = 0; c < 32; c += 4) {
-              float2 e0 = ffma2(make_float2(s[q * 32 + c], s[q * 32 + c + 1]), sl2x2, negm);
-              float2 e1 = ffma2(make_float2(s[q * 32 + c + 2], s[q * 32 + c + 3]), sl2x2, negm);
+              float2 e0 = ffma2(make_float2(S_(q * 32 + c), S_(q * 32 + c + 1)), sl2x2, negm);
+              float2 e1 = ffma2(make_float2(S_(q * 32 + c + 2), S_(q * 32 + c + 3)), sl2x2, negm);
               e0 = make_float2(ex2(e0.x), ex2(e0.y));
               e1 = make_float2(ex2(e1.x), ex2(e1.y));
               sum0 = fadd2(sum0, e0);
               sum1 = fadd2(sum1, e1);
-              pk[c / 2] = pack_bf16x2(e0.x, e0.y);
-              pk[c / 2 + 1] = pack_bf16x2(e1.x, e1.y);
+              pk[q * 16 + c / 2] = pack_bf16x2(e0.x, e0.y);
+              pk[q * 16 + c / 2 + 1] = pack_bf16x2(e1.x, e1.y);
             }
           } else {
 #pragma unroll
-            for (int c = 0; c < 16; ++c) pk[c] = 0u;
-          }
-          // P row -> shared memory, 128-byte swizzled K-major layout (16-byte chunk c of row r at c ^ (r & 7))
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int cc = q * 4 + u;  // 16-byte chunk index within the 128-byte row
-            *reinterpret_cast<uint4*>(prow + ((cc ^ sw) << 4)) =
-                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+            for (int c = 0; c < 16; ++c) pk[q * 16 + c] = 0u;
           }
         }
+#undef S_
         const float2 sum2 = fadd2(sum0, sum1);
         l_run += sum2.x + sum2.y;
-        fence_async_smem();
+        // P buffer g & 1 was last read by the PV of tile g - 2
+        if (g >= 2 && !wait_pv(g - 2)) { ok = false; break; }
+        tc_fence_after();
+        tmem_st32(lane_base + kPCol + (g & 1) * (kBN / 2), &pk[0]);
+        if (rescale) {
+          // scale O (the PV of the tiles before j, complete once PV(g - 1) is) for the rows whose
+          // reference max rose
+          if (g >= 1 && !wait_pv(g - 1)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int half = 0; half < 2; ++half) {
+            uint32_t o0[32];
+            tmem_ld32_sync(o_tmem + half * 32, o0);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o0[c] = __float_as_uint(__uint_as_float(o0[c]) * fscale);
+            tmem_st32(o_tmem + half * 32, o0);
+          }
+        }
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars->p_full[sb]);
+        mbar_arrive(&bars->p_full[g & 1]);
       }
       if (!ok) break;
-      // epilogue: the item's last PV, then O / l from TMEM
+      // epilogue: the item's last PV, then O / l from TMEM (the next item's first PV is
+      // issued only after this thread's next p_full arrival, so O is not overwritten early)
       if (!wait_pv(g - 1)) { ok = false; break; }
       tc_fence_after();
-      uint32_t o0[32], o1[32];
-      tmem_ld32_sync(o_tmem, o0);
-      tmem_ld32_sync(o_tmem + 32, o1);
-      tc_fence_before();
-      mbar_arrive(&bars->o_empty[ob]);
-      ++wi;
-      if (row_ok) {
-        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        uint4* dst = reinterpret_cast<uint4*>(O + ((tok0 + i) * H + it.h) * kDH);
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      const bool whole = it.q_last == it.q0 + kBM - 1;   // a full tile leaves through one TMA store
+      if (whole && n_stores > 0) {
+        // the staging tile is free once the previous store has read it
+        if (r == 0) {
+          tma_store_wait_read();
+          mbar_arrive(&bars->o_free);
+        }
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait_bounded(&bars->o_free, (n_stores - 1) & 1, abort_flag, kWaitNs))) {
+          ok = false;
+          break;
+        }
+      }
+      uint4* dst = reinterpret_cast<uint4*>(O + ((tok0 + i) * H + it.h) * kDH);
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        uint32_t o0[32];
+        tmem_ld32_sync(o_tmem + half * 32, o0);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint4 pk;
-          pk.x = pack_bf16x2(__uint_as_float(o0[c * 8 + 0]) * inv, __uint_as_float(o0[c * 8 + 1]) * inv);
-          pk.y = pack_bf16x2(__uint_as_float(o0[c * 8 + 2]) * inv, __uint_as_float(o0[c * 8 + 3]) * inv);
-          pk.z = pack_bf16x2(__uint_as_float(o0[c * 8 + 4]) * inv, __uint_as_float(o0[c * 8 + 5]) * inv);
-          pk.w = pack_bf16x2(__uint_as_float(o0[c * 8 + 6]) * inv, __uint_as_float(o0[c * 8 + 7]) * inv);
-          dst[c] = pk;
-          pk.x = pack_bf16x2(__uint_as_float(o1[c * 8 + 0]) * inv, __uint_as_float(o1[c * 8 + 1]) * inv);
-          pk.y = pack_bf16x2(__uint_as_float(o1[c * 8 + 2]) * inv, __uint_as_float(o1[c * 8 + 3]) * inv);
-          pk.z = pack_bf16x2(__uint_as_float(o1[c * 8 + 4]) * inv, __uint_as_float(o1[c * 8 + 5]) * inv);
-          pk.w = pack_bf16x2(__uint_as_float(o1[c * 8 + 6]) * inv, __uint_as_float(o1[c * 8 + 7]) * inv);
-          dst[4 + c] = pk;
+          uint4 pq;
+          pq.x = pack_bf16x2(__uint_as_float(o0[c * 8 + 0]) * inv, __uint_as_float(o0[c * 8 + 1]) * inv);
+          pq.y = pack_bf16x2(__uint_as_float(o0[c * 8 + 2]) * inv, __uint_as_float(o0[c * 8 + 3]) * inv);
+          pq.z = pack_bf16x2(__uint_as_float(o0[c * 8 + 4]) * inv, __uint_as_float(o0[c * 8 + 5]) * inv);
+          pq.w = pack_bf16x2(__uint_as_float(o0[c * 8 + 6]) * inv, __uint_as_float(o0[c * 8 + 7]) * inv);
+          const int cc = half * 4 + c;
+          // 128-byte swizzle of the staging tile (16-byte chunk cc of row r at cc ^ (r & 7))
+          if (whole) *reinterpret_cast<uint4*>(orow + ((cc ^ sw) << 4)) = pq;
+          else if (row_ok) dst[cc] = pq;
         }
-        if (a.lse)
-          a.lse[((int64_t)it.b * H + it.h) * n + i] = l_run > 0.f ? (m_ref + __log2f(l_run)) * kLn2 : -INFINITY;
       }
+      tc_fence_before();
+      if (whole) {
+        fence_async_smem();
+        mbar_arrive(&bars->o_ready);
+        if (warp == 0) {
+          // one thread issues the store once every row is in place; warp 0 leaves together on a timeout
+          bool okw = true;
+          if (lane == 0) {
+            okw = mbar_wait_bounded(&bars->o_ready, n_stores & 1, abort_flag, kWaitNs);
+            if (okw) tma_store_3d(&tm_o, smem + kOOff, 0, it.h, (int)(tok0 + it.q0));
+          }
+          if (!__shfl_sync(0xffffffffu, okw, 0)) {
+            ok = false;
+            break;
+          }
+        }
+        ++n_stores;
+      }
+      if (row_ok && a.lse)
+        a.lse[((int64_t)it.b * H + it.h) * n + i] = l_run > 0.f ? (m_ref + __log2f(l_run)) * kLn2 : -INFINITY;
     }
     if (!ok) {
       *abort_flag = 1;
       raise_status(a.status, ATTAMBA_DEV_TIMEOUT);
     }
+    // the stores must be complete before the CTA's shared memory goes away
+    if (r == 0 && n_stores > 0) tma_store_wait_all();
   }
 
   tc_fence_before();
@@ -581,8 +632,9 @@ bool encode_rows_map(CUtensorMap* m, const void* base, int64_t rows, int H, int 
 
 cudaError_t launch_chunk_attn_bf16(const AttnArgs& a, cudaStream_t s) {
   const int64_t T = (int64_t)a.B * a.n;
-  CUtensorMap tq, tk, tv, tkc, tvc;
-  if (!encode_rows_map(&tq, a.q, T, a.H, kBM) || !encode_rows_map(&tk, a.K, T, a.H, kBN) ||
+  CUtensorMap tq, tk, tv, tkc, tvc, to;
+  if (!encode_rows_map(&tq, a.q, T, a.H, kBM) || !encode_rows_map(&to, a.O, T, a.H, kBM) ||
+      !encode_rows_map(&tk, a.K, T, a.H, kBN) ||
       !encode_rows_map(&tv, a.V, T, a.H, kBN) || !encode_rows_map(&tkc, a.Kc, a.n_chunks, a.H, kBN) ||
       !encode_rows_map(&tvc, a.Vc, a.n_chunks, a.H, kBN))
     return cudaErrorNotSupported;
@@ -600,13 +652,13 @@ cudaError_t launch_chunk_attn_bf16(const AttnArgs& a, cudaStream_t s) {
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (sms <= 0) sms = 148;
   }
-  // persistent: one CTA per SM, each walking the work items (sequence, head, 128 queries) round robin;
-  // more CTAs only when an SM would hold more items than its table
+  // persistent: two CTAs per SM, each walking the work items (sequence, head, 128 queries) round
+  // robin; more CTAs only when a CTA would hold more items than its table
   const int64_t items = (int64_t)((a.n + kBM - 1) / kBM) * a.B * a.H;
   int64_t grid = items < (int64_t)kCtasPerSm * sms ? items : (int64_t)kCtasPerSm * sms;
   if ((items + grid - 1) / grid > kMaxItems) grid = (items + kMaxItems - 1) / kMaxItems;
   if (grid > 2147483647) return cudaErrorInvalidValue;
-  chunk_attn_bf16_kernel<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tkc, tvc, a);
+  chunk_attn_bf16_kernel<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tkc, tvc, to, a);
   return cudaGetLastError();
 }
 
