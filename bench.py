@@ -276,7 +276,9 @@ def decode_bench(dev, reps=3):
     return {"workload": cfg.name, "tokens_per_s": cfg.B * cfg.steps / (ms * 1e-3), "ms_per_step": per_step,
             "steps": cfg.steps, "batch": cfg.B, "context": cfg.ctx, "bytes_per_step": step_bytes,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                         "peak_source": f"{src} HBM copy"}, "gpu_launches_per_step": 3}
+                         "peak_source": f"{src} HBM copy", "traffic": ncu_traffic("decode_attn_kernel"),
+                         "traffic_kernel": "decode_attn_kernel"},
+            "gpu_launches_per_step": 3}
 
 
 # ------------------------------------------------------------------ CUDA path

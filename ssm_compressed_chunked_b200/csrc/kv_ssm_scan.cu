@@ -20,14 +20,17 @@
 //
 // The work is one exponential per (token, channel, state, SSM): 2 T D N of them
 // against 10 D bytes per token, so the multi-function unit (16 ex2 per clock
-// per SM), not HBM, sets the pace.  For bf16 outputs a share of the
-// exponentials (kPolyPairs of the N/2 pairs) runs on the FMA pipe instead:
-// 2^x = 2^j * 2^f with j = round(x) (added to the exponent field) and 2^f from
-// a degree-3 polynomial fitted here by the Remez exchange algorithm to the
+// per SM), not HBM, sets the pace; on the bench workload it is about 78% busy.
+// An FMA-pipe alternative is compiled in for bf16 outputs but off by default
+// (ATTAMBA_SCAN_POLY_PAIRS = 0): kPolyPairs of the N/2 state pairs would take
+// 2^x = 2^j * 2^f with j = round(x) (added to the exponent field) and 2^f from a
+// degree-3 polynomial fitted here by the Remez exchange algorithm to the
 // minimax relative error on [-1/2, 1/2] (max relative error 7.5e-5, far below
-// bf16's 2^-8).  The reduction is valid for x >= -125; a token where any lane
-// could go below uses the hardware exponential for every pair.  fp32 outputs
-// use the hardware exponential only.
+// bf16's 2^-8), valid for x >= -125 (a token where any lane could go below uses
+// the hardware exponential for every pair).  Measured on B200 every share of
+// it, like an FMA-pipe softplus or skipping the decay at chunk starts behind a
+// branch, was slower: the unit is busy, but the FMA pipe and the instruction
+// schedule (one basic block per token pair) are close behind.
 #include "common.cuh"
 #include "launch.h"
 
