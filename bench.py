@@ -407,7 +407,7 @@ def run_ours(args, ws, rank, local):
         ach = d["bytes"] / (d["ms"] * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
                 "peak_source": f"{src} HBM copy"}
-        roof["traffic"] = ncu_traffic("kv_ssm_scan_kernel" if dom == "kv_ssm_scan" else "query_index_kernel")
+        roof["traffic"] = ncu_traffic("kv_ssm_scan_kernel" if dom == "kv_ssm_scan" else "chunk_index_kernel")
     roof["kernel"] = dom
     scan = kernels["kv_ssm_scan"]
     out = {
