@@ -162,6 +162,28 @@ typedef struct {
   int32_t B, H, dh, N, P, offset, L, cap;
 } attamba_cache_t;
 
+/* attamba_cache_from_prefill -- the decode cache a prefill of positions [0, n0) leaves.
+ * [pith, core] at inference only the boundary states are cached; [pith, if] the
+ * final SSM state of each chunk, P = 8 with 64 leading tokens; [pith, carries] the
+ * leading-token window (Eq. 8).  Uniform chunks of the cache's P and offset.
+ *   cache     the cache to fill (its B, H, dh, N, P, offset, L, cap; device arrays).
+ *             Written: Kb, Vb, bpos rows 0..nb-1 (the positions p < n0 that end a
+ *             chunk, in order), the ring slots p mod L for p in [max(0, n0 - L), n0),
+ *             state (both SSMs after position n0 - 1: the recurrence rerun over the
+ *             tokens of the chunk holding n0 - 1), nb[b] = nb, pos[b] = n0.
+ *   K, V      [B, n0, H, dh] keys / values of the prefill (attamba_kv_ssm_scan).
+ *   x .. C_v  the prefill's scan inputs, token rows b * n0 + t, as in attamba_kv_ssm_scan.
+ *   n0        prefill length, >= 1.
+ * dtype ATTAMBA_BF16, dh 64, N 16, L >= 1.  ATTAMBA_ERR_INVALID_ARG when the
+ * boundaries of [0, n0) exceed cap (checked on the host: chunks are uniform). */
+attamba_status_t attamba_cache_from_prefill(attamba_dtype_t dtype, const attamba_cache_t* cache,
+                                            const void* K, const void* V, const void* x,
+                                            const void* dt_k, const void* dt_v, const float* bias_k,
+                                            const float* bias_v, const float* A_k, const float* A_v,
+                                            const void* B_k, const void* C_k, const void* B_v,
+                                            const void* C_v, int32_t n0, int32_t* d_status,
+                                            attamba_stream_t stream);
+
 /* Bytes of device workspace attamba_decode_step needs for this cache. */
 size_t attamba_decode_workspace_size(const attamba_cache_t* cache);
 

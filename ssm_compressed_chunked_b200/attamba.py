@@ -25,7 +25,7 @@ DEV_BAD_CHUNKS, DEV_CACHE_FULL, DEV_TIMEOUT = 0x1, 0x2, 0x4
 EXPORTS = ("attamba_version", "attamba_status_string", "attamba_last_error",
            "attamba_uniform_chunk_count", "attamba_chunk_index", "attamba_kv_ssm_scan",
            "attamba_chunk_attn_fwd", "attamba_decode_workspace_size", "attamba_decode_step",
-           "attamba_decode_step_noalloc")
+           "attamba_decode_step_noalloc", "attamba_cache_from_prefill")
 
 
 class AttambaError(RuntimeError):
@@ -78,6 +78,8 @@ def load():
                                      [f32, vp, vp, sz, vp, vp]
     L.attamba_decode_step_noalloc.restype = ctypes.c_int
     L.attamba_decode_step_noalloc.argtypes = [ctypes.c_int, ctypes.POINTER(CacheT)] + [vp] * 12 + [f32, vp, vp, vp]
+    L.attamba_cache_from_prefill.restype = ctypes.c_int
+    L.attamba_cache_from_prefill.argtypes = [ctypes.c_int, ctypes.POINTER(CacheT)] + [vp] * 13 + [i32, vp, vp]
     _lib = L
     return L
 
@@ -226,3 +228,19 @@ def decode_step_noalloc(cache, q_t, x_t, dt_k, dt_v, bias_k, bias_v, A_k, A_v, B
         _ptr(B_v, dt, "B_v"), _ptr(C_v, dt, "C_v"), float(scale), _ptr(o_t, dt, "o_t"),
         _ptr(status, torch.int32, "status", allow_none=True), _stream(stream))
     _check(st, "attamba_decode_step_noalloc")
+
+
+def cache_from_prefill(cache, K, V, x, dt_k, dt_v, bias_k, bias_v, A_k, A_v, B_k, C_k, B_v, C_v, n0,
+                       status=None, stream=None):
+    """attamba_cache_from_prefill: fill `cache` with what a prefill of positions [0, n0) of each
+    sequence leaves (boundary keys/values, the last L tokens, the SSM states after n0 - 1).
+    K, V: [B, n0, H, dh]; x, dt_k, dt_v: [B * n0, D]; B_k .. C_v: [B * n0, N] (bf16)."""
+    dt = torch.bfloat16
+    f32 = torch.float32
+    st = load().attamba_cache_from_prefill(
+        BF16, ctypes.byref(cache.c_struct()), _ptr(K, dt, "K"), _ptr(V, dt, "V"), _ptr(x, dt, "x"),
+        _ptr(dt_k, dt, "dt_k"), _ptr(dt_v, dt, "dt_v"), _ptr(bias_k, f32, "bias_k"), _ptr(bias_v, f32, "bias_v"),
+        _ptr(A_k, f32, "A_k"), _ptr(A_v, f32, "A_v"), _ptr(B_k, dt, "B_k"), _ptr(C_k, dt, "C_k"),
+        _ptr(B_v, dt, "B_v"), _ptr(C_v, dt, "C_v"), int(n0),
+        _ptr(status, torch.int32, "status", allow_none=True), _stream(stream))
+    _check(st, "attamba_cache_from_prefill")

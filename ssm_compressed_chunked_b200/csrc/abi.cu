@@ -168,6 +168,48 @@ attamba_status_t attamba_decode_step(attamba_dtype_t dtype, const attamba_cache_
   return e == cudaSuccess ? ATTAMBA_OK : cuda_fail(e, "attamba_decode_step");
 }
 
+attamba_status_t attamba_cache_from_prefill(attamba_dtype_t dtype, const attamba_cache_t* cache,
+                                            const void* K, const void* V, const void* x,
+                                            const void* dt_k, const void* dt_v, const float* bias_k,
+                                            const float* bias_v, const float* A_k, const float* A_v,
+                                            const void* B_k, const void* C_k, const void* B_v,
+                                            const void* C_v, int32_t n0, int32_t* d_status,
+                                            attamba_stream_t stream) {
+  (void)d_status;  // nothing is detected on the device: every limit is checked here
+  if (dtype != ATTAMBA_BF16) return ATTAMBA_ERR_UNSUPPORTED;
+  if (!cache) return ATTAMBA_ERR_INVALID_ARG;
+  const attamba_cache_t& c = *cache;
+  if (c.dh != 64 || c.N != 16) return ATTAMBA_ERR_UNSUPPORTED;
+  if (c.B < 1 || c.H < 1 || c.P < 1 || c.L < 1 || c.cap < 1 || n0 < 1) return ATTAMBA_ERR_INVALID_ARG;
+  if ((int64_t)c.B * c.H * c.cap * c.dh >= ((int64_t)1 << 40)) return ATTAMBA_ERR_INVALID_ARG;
+  if ((int64_t)c.B * n0 * c.H * c.dh >= ((int64_t)1 << 40)) return ATTAMBA_ERR_INVALID_ARG;
+  const void* req[] = {c.state, c.Kb, c.Vb, c.bpos, c.Kr, c.Vr, c.nb, c.pos, K, V, x, dt_k, dt_v,
+                       bias_k, bias_v, A_k, A_v, B_k, C_k, B_v, C_v};
+  for (const void* p : req)
+    if (!p) return ATTAMBA_ERR_INVALID_ARG;
+  const void* al[] = {c.Kb, c.Vb, c.Kr, c.Vr, K, V};
+  for (const void* p : al)
+    if (!aligned16(p)) return ATTAMBA_ERR_INVALID_ARG;
+  const int32_t nb = attamba::handoff_boundaries(n0, c.P, c.offset);
+  if (nb > c.cap) {
+    snprintf(g_err, sizeof(g_err), "attamba_cache_from_prefill: %d boundaries in [0, %d) exceed cap %d", nb, n0,
+             c.cap);
+    return ATTAMBA_ERR_INVALID_ARG;
+  }
+  attamba::HandoffArgs a{};
+  a.c = c;
+  a.K = K; a.V = V; a.x = x;
+  a.dt[0] = dt_k; a.dt[1] = dt_v;
+  a.bias[0] = bias_k; a.bias[1] = bias_v;
+  a.A[0] = A_k; a.A[1] = A_v;
+  a.Bm[0] = B_k; a.Bm[1] = B_v;
+  a.Cm[0] = C_k; a.Cm[1] = C_v;
+  a.n0 = n0;
+  a.nb = nb;
+  cudaError_t e = attamba::launch_cache_from_prefill(a, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTAMBA_OK : cuda_fail(e, "attamba_cache_from_prefill");
+}
+
 attamba_status_t attamba_decode_step_noalloc(attamba_dtype_t dtype, const attamba_cache_t* cache,
                                              const void* q_t, const void* x_t, const void* dt_k,
                                              const void* dt_v, const float* bias_k, const float* bias_v,

@@ -71,4 +71,21 @@ size_t decode_noalloc_scratch_bytes();
 cudaError_t decode_noalloc_scratch(float** out);
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s);
 
+struct HandoffArgs {
+  attamba_cache_t c;
+  const void* K;
+  const void* V;
+  const void* x;
+  const void* dt[2];
+  const float* bias[2];
+  const float* A[2];
+  const void* Bm[2];
+  const void* Cm[2];
+  int32_t n0;
+  int32_t nb;   // boundaries in [0, n0)
+};
+// number of positions p < n0 that end a uniform chunk (size P, offset)
+int32_t handoff_boundaries(int32_t n0, int32_t P, int32_t offset);
+cudaError_t launch_cache_from_prefill(const HandoffArgs& a, cudaStream_t s);
+
 }  // namespace attamba

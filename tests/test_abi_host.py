@@ -69,6 +69,13 @@ def test_invalid_arguments_are_rejected_on_the_host():
     assert lib.attamba_decode_step(0, ctypes.byref(c), *([fake] * 12), ctypes.c_float(0.1), fake, fake,
                                    1 << 20, None, None) == A.ERR_UNSUPPORTED
     assert lib.attamba_decode_workspace_size(ctypes.byref(c)) > 0
+    # prefill -> cache handoff: f32, empty prefill, more boundaries than the cache holds
+    c.cap = 3
+    args = [fake] * 13
+    assert lib.attamba_cache_from_prefill(0, ctypes.byref(c), *args, 64, None, None) == A.ERR_UNSUPPORTED
+    assert lib.attamba_cache_from_prefill(1, ctypes.byref(c), *args, 0, None, None) == A.ERR_INVALID_ARG
+    assert lib.attamba_cache_from_prefill(1, ctypes.byref(c), *args, 64, None, None) == A.ERR_INVALID_ARG
+    assert b"exceed cap" in lib.attamba_last_error()
 
 
 def test_cpu_tensors_are_refused():
