@@ -133,6 +133,20 @@ attamba_status_t attamba_kv_ssm_scan(attamba_dtype_t dtype, const void* x, const
                                      int32_t N, void* K, void* V, void* Kc, void* Vc,
                                      int32_t* d_status, attamba_stream_t stream);
 
+/* attamba_kv_ssm_scan_u -- attamba_kv_ssm_scan with a separate input per SSM: the
+ * keys SSM reads u_k, the values SSM u_v.  This is the kept-projection variant
+ * [pith, if] (removing the explicit K and V projections costs about 1%, so with
+ * them kept the SSM input is u = x W_K for the keys and u = x W_V for the values);
+ * the projections are the caller's, as for q.  Same arguments, layouts, limits and
+ * errors as attamba_kv_ssm_scan otherwise; u_k == u_v is the shared-input case. */
+attamba_status_t attamba_kv_ssm_scan_u(attamba_dtype_t dtype, const void* u_k, const void* u_v,
+                                       const void* dt_k, const void* dt_v, const float* bias_k,
+                                       const float* bias_v, const float* A_k, const float* A_v,
+                                       const void* B_k, const void* C_k, const void* B_v, const void* C_v,
+                                       const int32_t* cu, int32_t n_chunks, int64_t T, int32_t D, int32_t N,
+                                       void* K, void* V, void* Kc, void* Vc, int32_t* d_status,
+                                       attamba_stream_t stream);
+
 /* attamba_chunk_attn_fwd -- softmax attention of every query over its key set S(i).
  * [pith, carries] (attention map (n/P + L) x (n/P + L)), [pith, core].
  *   q, K, V   [T, H, dh] (T = idx->B * idx->n);  Kc, Vc [idx->n_chunks, H, dh].

@@ -25,7 +25,8 @@ DEV_BAD_CHUNKS, DEV_CACHE_FULL, DEV_TIMEOUT = 0x1, 0x2, 0x4
 EXPORTS = ("attamba_version", "attamba_status_string", "attamba_last_error",
            "attamba_uniform_chunk_count", "attamba_chunk_index", "attamba_kv_ssm_scan",
            "attamba_chunk_attn_fwd", "attamba_decode_workspace_size", "attamba_decode_step",
-           "attamba_decode_step_noalloc", "attamba_cache_from_prefill")
+           "attamba_decode_step_noalloc", "attamba_cache_from_prefill",
+           "attamba_kv_ssm_scan_u")
 
 
 class AttambaError(RuntimeError):
@@ -68,6 +69,8 @@ def load():
                                       ctypes.POINTER(IndexT), vp, vp]
     L.attamba_kv_ssm_scan.restype = ctypes.c_int
     L.attamba_kv_ssm_scan.argtypes = [ctypes.c_int] + [vp] * 12 + [i32, i64, i32, i32] + [vp] * 4 + [vp, vp]
+    L.attamba_kv_ssm_scan_u.restype = ctypes.c_int
+    L.attamba_kv_ssm_scan_u.argtypes = [ctypes.c_int] + [vp] * 13 + [i32, i64, i32, i32] + [vp] * 4 + [vp, vp]
     L.attamba_chunk_attn_fwd.restype = ctypes.c_int
     L.attamba_chunk_attn_fwd.argtypes = [ctypes.c_int, vp, vp, vp, vp, vp, ctypes.POINTER(IndexT),
                                          i32, i32, f32, vp, vp, vp, vp]
@@ -165,6 +168,26 @@ def kv_ssm_scan(x, dt_k, dt_v, bias_k, bias_v, A_k, A_v, B_k, C_k, B_v, C_v, cu,
         _ptr(Kc, dt, "Kc", allow_none=True), _ptr(Vc, dt, "Vc", allow_none=True),
         _ptr(status, torch.int32, "status", allow_none=True), _stream(stream))
     _check(st, "attamba_kv_ssm_scan")
+
+
+def kv_ssm_scan_u(u_k, u_v, dt_k, dt_v, bias_k, bias_v, A_k, A_v, B_k, C_k, B_v, C_v, cu, n_chunks, K, V,
+                  Kc=None, Vc=None, status=None, stream=None):
+    """attamba_kv_ssm_scan_u: the keys SSM reads u_k, the values SSM u_v (kept-projection variant)."""
+    dt = u_k.dtype
+    D = u_k.shape[-1]
+    T = u_k.numel() // D
+    N = A_k.shape[-1]
+    f32 = torch.float32
+    if u_v.shape != u_k.shape:
+        raise AttambaError("u_k and u_v must have the same shape")
+    st = load().attamba_kv_ssm_scan_u(
+        _dtype_code(u_k), _ptr(u_k, dt, "u_k"), _ptr(u_v, dt, "u_v"), _ptr(dt_k, dt, "dt_k"), _ptr(dt_v, dt, "dt_v"),
+        _ptr(bias_k, f32, "bias_k"), _ptr(bias_v, f32, "bias_v"), _ptr(A_k, f32, "A_k"), _ptr(A_v, f32, "A_v"),
+        _ptr(B_k, dt, "B_k"), _ptr(C_k, dt, "C_k"), _ptr(B_v, dt, "B_v"), _ptr(C_v, dt, "C_v"),
+        _ptr(cu, torch.int32, "cu"), n_chunks, T, D, N, _ptr(K, dt, "K"), _ptr(V, dt, "V"),
+        _ptr(Kc, dt, "Kc", allow_none=True), _ptr(Vc, dt, "Vc", allow_none=True),
+        _ptr(status, torch.int32, "status", allow_none=True), _stream(stream))
+    _check(st, "attamba_kv_ssm_scan_u")
 
 
 def chunk_attn_fwd(q, K, V, Kc, Vc, index, scale, O, lse=None, status=None, stream=None):

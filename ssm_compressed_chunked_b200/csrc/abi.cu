@@ -63,6 +63,42 @@ attamba_status_t attamba_chunk_index(const int32_t* cu_in, int32_t n_chunks, int
   return e == cudaSuccess ? ATTAMBA_OK : cuda_fail(e, "attamba_chunk_index");
 }
 
+namespace {
+attamba_status_t scan_entry(attamba_dtype_t dtype, const void* u_k, const void* u_v, const void* dt_k,
+                            const void* dt_v, const float* bias_k, const float* bias_v, const float* A_k,
+                            const float* A_v, const void* B_k, const void* C_k, const void* B_v, const void* C_v,
+                            const int32_t* cu, int32_t n_chunks, int64_t T, int32_t D, int32_t N, void* K,
+                            void* V, void* Kc, void* Vc, int32_t* d_status, cudaStream_t stream, const char* name) {
+  if (!ok_dtype(dtype)) return ATTAMBA_ERR_UNSUPPORTED;
+  if (N != 16) return ATTAMBA_ERR_UNSUPPORTED;
+  if (T < 1 || T >= kMaxTokens || D < 8 || D % 8 != 0 || n_chunks < 1 || n_chunks > T)
+    return ATTAMBA_ERR_INVALID_ARG;
+  if (T * D >= kMaxTokens) return ATTAMBA_ERR_UNSUPPORTED;  // element offsets are 32-bit
+  const void* req[] = {u_k, u_v, dt_k, dt_v, bias_k, bias_v, A_k, A_v, B_k, C_k, B_v, C_v, cu, K, V};
+  for (const void* p : req)
+    if (!p || !aligned16(p)) return ATTAMBA_ERR_INVALID_ARG;
+  if ((Kc == nullptr) != (Vc == nullptr)) return ATTAMBA_ERR_INVALID_ARG;
+  if (Kc && (!aligned16(Kc) || !aligned16(Vc))) return ATTAMBA_ERR_INVALID_ARG;
+  attamba::ScanArgs a{};
+  a.x[0] = u_k; a.x[1] = u_v;
+  a.dt[0] = dt_k; a.dt[1] = dt_v;
+  a.bias[0] = bias_k; a.bias[1] = bias_v;
+  a.A[0] = A_k; a.A[1] = A_v;
+  a.Bm[0] = B_k; a.Bm[1] = B_v;
+  a.Cm[0] = C_k; a.Cm[1] = C_v;
+  a.cu = cu;
+  a.n_chunks = n_chunks;
+  a.T = T;
+  a.D = D;
+  a.N = N;
+  a.out[0] = K; a.out[1] = V;
+  a.outc[0] = Kc; a.outc[1] = Vc;
+  a.status = d_status;
+  cudaError_t e = attamba::launch_kv_ssm_scan(dtype, a, stream);
+  return e == cudaSuccess ? ATTAMBA_OK : cuda_fail(e, name);
+}
+}  // namespace
+
 attamba_status_t attamba_kv_ssm_scan(attamba_dtype_t dtype, const void* x, const void* dt_k,
                                      const void* dt_v, const float* bias_k, const float* bias_v,
                                      const float* A_k, const float* A_v, const void* B_k,
@@ -70,29 +106,19 @@ attamba_status_t attamba_kv_ssm_scan(attamba_dtype_t dtype, const void* x, const
                                      const int32_t* cu, int32_t n_chunks, int64_t T, int32_t D,
                                      int32_t N, void* K, void* V, void* Kc, void* Vc,
                                      int32_t* d_status, attamba_stream_t stream) {
-  if (!ok_dtype(dtype)) return ATTAMBA_ERR_UNSUPPORTED;
-  if (N != 16) return ATTAMBA_ERR_UNSUPPORTED;
-  if (T < 1 || T >= kMaxTokens || D < 8 || D % 8 != 0 || n_chunks < 1 || n_chunks > T)
-    return ATTAMBA_ERR_INVALID_ARG;
-  if (T * D >= kMaxTokens) return ATTAMBA_ERR_UNSUPPORTED;  // element offsets are 32-bit
-  const void* req[] = {x, dt_k, dt_v, bias_k, bias_v, A_k, A_v, B_k, C_k, B_v, C_v, cu, K, V};
-  for (const void* p : req)
-    if (!p || !aligned16(p)) return ATTAMBA_ERR_INVALID_ARG;
-  if ((Kc == nullptr) != (Vc == nullptr)) return ATTAMBA_ERR_INVALID_ARG;
-  if (Kc && (!aligned16(Kc) || !aligned16(Vc))) return ATTAMBA_ERR_INVALID_ARG;
-  attamba::ScanArgs a{};
-  a.x = x;
-  a.dt[0] = dt_k; a.dt[1] = dt_v;
-  a.bias[0] = bias_k; a.bias[1] = bias_v;
-  a.A[0] = A_k; a.A[1] = A_v;
-  a.Bm[0] = B_k; a.Bm[1] = B_v;
-  a.Cm[0] = C_k; a.Cm[1] = C_v;
-  a.cu = cu; a.n_chunks = n_chunks; a.T = T; a.D = D; a.N = N;
-  a.out[0] = K; a.out[1] = V;
-  a.outc[0] = Kc; a.outc[1] = Vc;
-  a.status = d_status;
-  cudaError_t e = attamba::launch_kv_ssm_scan(dtype, a, reinterpret_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? ATTAMBA_OK : cuda_fail(e, "attamba_kv_ssm_scan");
+  return scan_entry(dtype, x, x, dt_k, dt_v, bias_k, bias_v, A_k, A_v, B_k, C_k, B_v, C_v, cu, n_chunks, T, D, N,
+                    K, V, Kc, Vc, d_status, reinterpret_cast<cudaStream_t>(stream), "attamba_kv_ssm_scan");
+}
+
+attamba_status_t attamba_kv_ssm_scan_u(attamba_dtype_t dtype, const void* u_k, const void* u_v,
+                                       const void* dt_k, const void* dt_v, const float* bias_k,
+                                       const float* bias_v, const float* A_k, const float* A_v,
+                                       const void* B_k, const void* C_k, const void* B_v, const void* C_v,
+                                       const int32_t* cu, int32_t n_chunks, int64_t T, int32_t D, int32_t N,
+                                       void* K, void* V, void* Kc, void* Vc, int32_t* d_status,
+                                       attamba_stream_t stream) {
+  return scan_entry(dtype, u_k, u_v, dt_k, dt_v, bias_k, bias_v, A_k, A_v, B_k, C_k, B_v, C_v, cu, n_chunks, T, D,
+                    N, K, V, Kc, Vc, d_status, reinterpret_cast<cudaStream_t>(stream), "attamba_kv_ssm_scan_u");
 }
 
 attamba_status_t attamba_chunk_attn_fwd(attamba_dtype_t dtype, const void* q, const void* K,

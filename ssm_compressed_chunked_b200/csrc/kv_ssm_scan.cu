@@ -201,7 +201,7 @@ __global__ void __launch_bounds__(kScanThreads, ATTAMBA_SCAN_MINB) kv_ssm_scan_k
   const int32_t c_end = min(c_begin + chunks_per_block, p.n_chunks);
   for (int i = threadIdx.x; i <= c_end - c_begin; i += kScanThreads) sCu[i] = p.cu[c_begin + i];
 
-  const T* __restrict__ x = static_cast<const T*>(p.x) + d0;
+  const T* __restrict__ x = static_cast<const T*>(p.x[s]) + d0;
   const T* __restrict__ dt = static_cast<const T*>(p.dt[s]) + d0;
   const T* __restrict__ Bm = static_cast<const T*>(p.Bm[s]);
   const T* __restrict__ Cm = static_cast<const T*>(p.Cm[s]);

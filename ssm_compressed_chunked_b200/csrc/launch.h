@@ -13,7 +13,7 @@ cudaError_t launch_chunk_index(const int32_t* cu_in, int32_t n_chunks, int32_t B
                                const attamba_index_t& out, int32_t* d_status, cudaStream_t s);
 
 struct ScanArgs {
-  const void* x;
+  const void* x[2];   // SSM input of the keys SSM and of the values SSM (the same array unless kept projections)
   const void* dt[2];
   const float* bias[2];
   const float* A[2];

@@ -56,3 +56,45 @@ def test_scan_full_size_sampled_chunks(ci):
             assert_close(cfg.dtype, f64(K[b, t0:t1]), rk, f"K b={b} chunk={c}")
             assert_close(cfg.dtype, f64(V[b, t0:t1]), rv, f"V b={b} chunk={c}")
     assert pf.status.item() == 0
+
+
+@pytest.mark.parametrize("cfg", [W.shrink(W.LAYER_CONFIGS[1], B=2, n=300, D=128, H=2),
+                                 W.shrink(W.LAYER_CONFIGS[0], B=2, n=77, D=64, H=1, P=16, offset=5)],
+                         ids=lambda c: f"{c.name}-n{c.n}-D{c.D}")
+def test_scan_kept_projection_inputs(cfg):
+    """attamba_kv_ssm_scan_u: the keys SSM reads u_k = x W_K, the values SSM u_v = x W_V (the
+    kept-projection variant); each must match the oracle recurrence over its own input, and u_k = u_v = x
+    must reproduce attamba_kv_ssm_scan bit for bit."""
+    from ssm_compressed_chunked_b200 import attamba as A, layer
+    from oracle import ssm as OS
+    inp = W.make_layer(cfg)
+    pf = run_prefill(inp, cfg)
+    g = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    gen = torch.Generator().manual_seed(11)
+    dt = W.torch_dtype(cfg.dtype)
+    proj = [torch.randn(cfg.D, cfg.D, generator=gen) / cfg.D ** 0.5 for _ in range(2)]
+    x32 = inp["x"].float().reshape(-1, cfg.D)
+    u = [(x32 @ w).to(dt) for w in proj]                     # the caller's projections, rounded like q
+    T = cfg.B * cfg.n
+    K = torch.empty(T, cfg.D, dtype=dt, device="cuda")
+    V = torch.empty_like(K)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    flat = lambda t: t.reshape(T, -1)
+    args = (flat(g["dt_k"]), flat(g["dt_v"]), g["bias_k"], g["bias_v"], g["A_k"], g["A_v"], flat(g["B_k"]),
+            flat(g["C_k"]), flat(g["B_v"]), flat(g["C_v"]), pf.index.cu, pf.n_chunks)
+    A.kv_ssm_scan_u(u[0].cuda(), u[1].cuda(), *args, K, V, status=status)
+    # shared input through the new entry point equals the original one exactly
+    K2 = torch.empty_like(K)
+    V2 = torch.empty_like(K)
+    A.kv_ssm_scan_u(flat(g["x"]), flat(g["x"]), *args, K2, V2, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.equal(K2, pf.K) and torch.equal(V2, pf.V)
+    for b in range(cfg.B):
+        is_start = OC.is_start_mask(np.asarray(inp["starts"][b]), cfg.n)
+        sl = slice(b * cfg.n, (b + 1) * cfg.n)
+        for s, name, out in ((0, "k", K), (1, "v", V)):
+            ref, _ = OS.selective_scan(f64(u[s][sl]), f64(inp["dt_" + name][b]), f64(inp["bias_" + name]),
+                                       f64(inp["A_" + name]), f64(inp["B_" + name][b]), f64(inp["C_" + name][b]),
+                                       is_start)
+            assert_close(cfg.dtype, f64(out[sl]), ref, f"{name} b={b}")
