@@ -120,7 +120,7 @@ attamba_status_t attamba_chunk_index(const int32_t* cu_in, int32_t n_chunks, int
  *   bias_k/v  [D] f32;  A_k/v [D, N] f32 (negative).
  *   B_k, C_k, B_v, C_v   [T, N].
  *   cu        [n_chunks+1] chunk starts (as written by attamba_chunk_index).
- *   N         16 (supported state size);  D a multiple of 8.
+ *   N         16 or 32 (the supported state sizes; 32 is the pages' default Ds)  D a multiple of 8.
  *   K, V      [T, D] outputs (viewed as [T, H, dh] by the attention).
  *   Kc, Vc    nullable [n_chunks, D]: K, V at the last token of each chunk (the
  *             boundary states), the compact copy the attention reads.
@@ -188,7 +188,7 @@ typedef struct {
  *   K, V      [B, n0, H, dh] keys / values of the prefill (attamba_kv_ssm_scan).
  *   x .. C_v  the prefill's scan inputs, token rows b * n0 + t, as in attamba_kv_ssm_scan.
  *   n0        prefill length, >= 1.
- * dtype ATTAMBA_BF16, dh 64, N 16, L >= 1.  ATTAMBA_ERR_INVALID_ARG when the
+ * dtype ATTAMBA_BF16, dh 64, N 16 or 32, L >= 1.  ATTAMBA_ERR_INVALID_ARG when the
  * boundaries of [0, n0) exceed cap (checked on the host: chunks are uniform). */
 attamba_status_t attamba_cache_from_prefill(attamba_dtype_t dtype, const attamba_cache_t* cache,
                                             const void* K, const void* V, const void* x,
@@ -210,7 +210,7 @@ size_t attamba_decode_workspace_size(const attamba_cache_t* cache);
  * them to the boundary list (ATTAMBA_DEV_CACHE_FULL if nb == cap); then attend
  * q_t over { boundaries at positions < t-L+1 } united with [t-L+1, t].  Finally
  * pos[b] += 1 and nb[b] grows by the append.
- *   dtype      ATTAMBA_BF16 (the cache and the step tensors);  L >= 1, dh = 64, N = 16.
+ *   dtype      ATTAMBA_BF16 (the cache and the step tensors);  L >= 1, dh = 64, N = 16 or 32.
  *   q_t        [B, H, dh];  x_t, dt_k, dt_v [B, D];  B_k, C_k, B_v, C_v [B, N].
  *   bias_*, A_* as in attamba_kv_ssm_scan.
  *   o_t        [B, H, dh] output.

@@ -70,7 +70,7 @@ attamba_status_t scan_entry(attamba_dtype_t dtype, const void* u_k, const void* 
                             const int32_t* cu, int32_t n_chunks, int64_t T, int32_t D, int32_t N, void* K,
                             void* V, void* Kc, void* Vc, int32_t* d_status, cudaStream_t stream, const char* name) {
   if (!ok_dtype(dtype)) return ATTAMBA_ERR_UNSUPPORTED;
-  if (N != 16) return ATTAMBA_ERR_UNSUPPORTED;
+  if (N != 16 && N != 32) return ATTAMBA_ERR_UNSUPPORTED;
   if (T < 1 || T >= kMaxTokens || D < 8 || D % 8 != 0 || n_chunks < 1 || n_chunks > T)
     return ATTAMBA_ERR_INVALID_ARG;
   if (T * D >= kMaxTokens) return ATTAMBA_ERR_UNSUPPORTED;  // element offsets are 32-bit
@@ -166,7 +166,7 @@ attamba_status_t attamba_decode_step(attamba_dtype_t dtype, const attamba_cache_
   if (dtype != ATTAMBA_BF16) return ATTAMBA_ERR_UNSUPPORTED;
   if (!cache) return ATTAMBA_ERR_INVALID_ARG;
   const attamba_cache_t& c = *cache;
-  if (c.dh != 64 || c.N != 16) return ATTAMBA_ERR_UNSUPPORTED;
+  if (c.dh != 64 || (c.N != 16 && c.N != 32)) return ATTAMBA_ERR_UNSUPPORTED;
   if (c.B < 1 || c.H < 1 || c.P < 1 || c.L < 1 || c.cap < 1) return ATTAMBA_ERR_INVALID_ARG;
   if ((int64_t)c.B * c.H * c.cap * c.dh >= ((int64_t)1 << 40)) return ATTAMBA_ERR_INVALID_ARG;
   const void* req[] = {c.state, c.Kb, c.Vb, c.bpos, c.Kr, c.Vr, c.nb, c.pos, q_t, x_t, dt_k, dt_v,
@@ -205,7 +205,7 @@ attamba_status_t attamba_cache_from_prefill(attamba_dtype_t dtype, const attamba
   if (dtype != ATTAMBA_BF16) return ATTAMBA_ERR_UNSUPPORTED;
   if (!cache) return ATTAMBA_ERR_INVALID_ARG;
   const attamba_cache_t& c = *cache;
-  if (c.dh != 64 || c.N != 16) return ATTAMBA_ERR_UNSUPPORTED;
+  if (c.dh != 64 || (c.N != 16 && c.N != 32)) return ATTAMBA_ERR_UNSUPPORTED;
   if (c.B < 1 || c.H < 1 || c.P < 1 || c.L < 1 || c.cap < 1 || n0 < 1) return ATTAMBA_ERR_INVALID_ARG;
   if ((int64_t)c.B * c.H * c.cap * c.dh >= ((int64_t)1 << 40)) return ATTAMBA_ERR_INVALID_ARG;
   if ((int64_t)c.B * n0 * c.H * c.dh >= ((int64_t)1 << 40)) return ATTAMBA_ERR_INVALID_ARG;
@@ -246,7 +246,7 @@ attamba_status_t attamba_decode_step_noalloc(attamba_dtype_t dtype, const attamb
   if (dtype != ATTAMBA_BF16) return ATTAMBA_ERR_UNSUPPORTED;
   if (!cache) return ATTAMBA_ERR_INVALID_ARG;
   const attamba_cache_t& c = *cache;
-  if (c.dh != 64 || c.N != 16) return ATTAMBA_ERR_UNSUPPORTED;
+  if (c.dh != 64 || (c.N != 16 && c.N != 32)) return ATTAMBA_ERR_UNSUPPORTED;
   if (c.B < 1 || c.H < 1 || c.P < 1 || c.L < 1 || c.cap < 1) return ATTAMBA_ERR_INVALID_ARG;
   if ((int64_t)c.B * c.H * c.cap * c.dh >= ((int64_t)1 << 40)) return ATTAMBA_ERR_INVALID_ARG;
   const void* req[] = {c.state, c.Kb, c.Vb, c.bpos, c.Kr, c.Vr, c.nb, c.pos, q_t, x_t, dt_k, dt_v,

@@ -38,7 +38,6 @@ static __device__ __align__(256) float g_decode_scratch[kNoAllocScratchFloats];
 
 namespace {
 constexpr int kDH = 64;
-constexpr int kNS = 16;
 constexpr int kAttnThreads = 128;
 constexpr int kUnroll = 4;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -50,6 +49,7 @@ __device__ __forceinline__ bool chunk_ends_at(int t, int P, int o) {
   return (t + 1 >= o) && ((t + 1 - o) % P == 0);
 }
 
+template <int kNS>
 __global__ void __launch_bounds__(128) decode_ssm_kernel(DecodeArgs a) {
   const attamba_cache_t& c = a.c;
   const int D = c.H * c.dh;
@@ -329,7 +329,10 @@ size_t decode_workspace_bytes(const attamba_cache_t& c) {
 
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s) {
   const int D = a.c.H * a.c.dh;
-  decode_ssm_kernel<<<dim3((D + 127) / 128, a.c.B, 2), 128, 0, s>>>(a);
+  if (a.c.N == 32)
+    decode_ssm_kernel<32><<<dim3((D + 127) / 128, a.c.B, 2), 128, 0, s>>>(a);
+  else
+    decode_ssm_kernel<16><<<dim3((D + 127) / 128, a.c.B, 2), 128, 0, s>>>(a);
   decode_attn_kernel<<<dim3(a.splits, a.c.H, a.c.B), kAttnThreads, 0, s>>>(a);
   decode_combine_kernel<<<a.c.B * a.c.H, kDH, 0, s>>>(a);
   return cudaGetLastError();

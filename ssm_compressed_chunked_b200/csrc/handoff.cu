@@ -20,7 +20,6 @@ namespace attamba {
 
 namespace {
 constexpr int kDH = 64;
-constexpr int kNS = 16;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // one past the first chunk end of a uniform chunking: the offset mod P, or P when that is 0
@@ -61,6 +60,7 @@ __global__ void __launch_bounds__(128) handoff_copy_kernel(HandoffArgs a) {
 }
 
 // thread (s, b, d): the SSM state after position n0 - 1, rerun from the start of its chunk
+template <int kNS>
 __global__ void __launch_bounds__(128) handoff_state_kernel(HandoffArgs a) {
   const attamba_cache_t& c = a.c;
   const int D = c.H * c.dh;
@@ -104,7 +104,10 @@ cudaError_t launch_cache_from_prefill(const HandoffArgs& a, cudaStream_t s) {
   const int nring = a.c.L < a.n0 ? a.c.L : a.n0;
   handoff_copy_kernel<<<dim3(a.nb + nring, a.c.B), 128, 0, s>>>(a);
   const int D = a.c.H * a.c.dh;
-  handoff_state_kernel<<<dim3((D + 127) / 128, a.c.B, 2), 128, 0, s>>>(a);
+  if (a.c.N == 32)
+    handoff_state_kernel<32><<<dim3((D + 127) / 128, a.c.B, 2), 128, 0, s>>>(a);
+  else
+    handoff_state_kernel<16><<<dim3((D + 127) / 128, a.c.B, 2), 128, 0, s>>>(a);
   return cudaGetLastError();
 }
 

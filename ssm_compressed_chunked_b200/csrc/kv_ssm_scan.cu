@@ -53,8 +53,6 @@ constexpr int kScanThreads = 128;
 #endif
 constexpr int kStageTokens = 64;       // B/C staging window (even, so token pairs never straddle one)
 constexpr int kMaxChunksPerBlock = 256;
-constexpr int kNS = 16;
-constexpr int kNP = kNS / 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kPolyMinExp = -125.f;
 // 2^f on [-1/2, 1/2], minimax relative error (own Remez fit), f32 coefficients
@@ -133,6 +131,18 @@ template <> struct Vec<__nv_bfloat16, 2> {
     *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v[0], v[1]);
   }
 };
+template <> struct Vec<__nv_bfloat16, 1> {
+  using raw = unsigned short;
+  static __device__ __forceinline__ raw load(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const unsigned short*>(p)); }
+  static __device__ __forceinline__ void unpack(raw r, float (&v)[1]) { v[0] = __uint_as_float((uint32_t)r << 16); }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[1]) { *p = __float2bfloat16_rn(v[0]); }
+};
+template <> struct Vec<float, 1> {
+  using raw = float;
+  static __device__ __forceinline__ raw load(const float* p) { return __ldg(p); }
+  static __device__ __forceinline__ void unpack(raw r, float (&v)[1]) { v[0] = r; }
+  static __device__ __forceinline__ void store(float* p, const float (&v)[1]) { *p = v[0]; }
+};
 template <> struct Vec<float, 2> {
   using raw = float2;
   static __device__ __forceinline__ raw load(const float* p) { return __ldg(reinterpret_cast<const float2*>(p)); }
@@ -142,8 +152,9 @@ template <> struct Vec<float, 2> {
   }
 };
 
-// Per-thread state of the scan: CPT channels x N/2 state pairs.
-template <int CPT> struct ScanState {
+// Per-thread state of the scan: CPT channels x NS/2 state pairs.
+template <int CPT, int NS> struct ScanState {
+  static constexpr int kNP = NS / 2;
   float2 a2[CPT][kNP];  // A * log2 e
   float2 h[CPT][kNP];
   float bias[CPT];
@@ -153,9 +164,10 @@ template <int CPT> struct ScanState {
 // One token: decay, input, readout.  `reset` marks a chunk start: its delta in
 // the exponent is replaced by a huge value so exp(delta A) = 0 (A < 0) and the
 // state restarts from the token's own input, with no branch.
-template <typename T, int CPT, int POLY_PAIRS>
-__device__ __forceinline__ void scan_token(ScanState<CPT>& st, const float* __restrict__ bc, const float (&dl)[CPT],
+template <typename T, int CPT, int NS, int POLY_PAIRS>
+__device__ __forceinline__ void scan_token(ScanState<CPT, NS>& st, const float* __restrict__ bc, const float (&dl)[CPT],
                                            const float (&dx)[CPT], bool reset, bool poly_ok, float (&y)[CPT]) {
+  constexpr int kNP = NS / 2;
   const float4* bc4 = reinterpret_cast<const float4*>(bc);
   float2 Bp[kNP], Cp[kNP];
 #pragma unroll
@@ -186,9 +198,11 @@ __device__ __forceinline__ void scan_token(ScanState<CPT>& st, const float* __re
   }
 }
 
-template <typename T, int CPT, int POLY_PAIRS>
-__global__ void __launch_bounds__(kScanThreads, ATTAMBA_SCAN_MINB) kv_ssm_scan_kernel(ScanArgs p, int32_t chunks_per_block) {
+template <typename T, int CPT, int NS, int POLY_PAIRS, int MINB>
+__global__ void __launch_bounds__(kScanThreads, MINB) kv_ssm_scan_kernel(ScanArgs p, int32_t chunks_per_block) {
   using V = Vec<T, CPT>;
+  constexpr int kNS = NS;
+  constexpr int kNP = NS / 2;
   __shared__ __align__(16) float sBC[kStageTokens][2 * kNS];  // B then C of each staged token
   __shared__ int sCu[kMaxChunksPerBlock + 1];                 // chunk starts of this block
 
@@ -208,7 +222,7 @@ __global__ void __launch_bounds__(kScanThreads, ATTAMBA_SCAN_MINB) kv_ssm_scan_k
   T* __restrict__ out = static_cast<T*>(p.out[s]) + d0;
   T* __restrict__ outc = static_cast<T*>(p.outc[s]);
 
-  ScanState<CPT> st;
+  ScanState<CPT, NS> st;
   st.amax = 0.f;
 #pragma unroll
   for (int c = 0; c < CPT; ++c) {
@@ -261,7 +275,7 @@ __global__ void __launch_bounds__(kScanThreads, ATTAMBA_SCAN_MINB) kv_ssm_scan_k
     bool poly_ok = false;
     if (POLY_PAIRS > 0) poly_ok = !reset && !__any_sync(__activemask(), dmax * st.amax > -kPolyMinExp);
     float y[CPT];
-    scan_token<T, CPT, POLY_PAIRS>(st, bc, dl, dx, reset, poly_ok, y);
+    scan_token<T, CPT, NS, POLY_PAIRS>(st, bc, dl, dx, reset, poly_ok, y);
     V::store(out + t * D, y);
     if (outc != nullptr && t + 1 == next_start) V::store(outc + (c_begin + ci) * D + d0, y);
   };
@@ -290,8 +304,10 @@ __global__ void __launch_bounds__(kScanThreads, ATTAMBA_SCAN_MINB) kv_ssm_scan_k
 }
 }  // namespace
 
-cudaError_t launch_kv_ssm_scan(attamba_dtype_t dtype, const ScanArgs& a, cudaStream_t s) {
-  constexpr int CPT = ATTAMBA_SCAN_CPT;
+namespace {
+// N = 16: two channels per thread; N = 32: one (the state and A of two channels would not fit)
+template <int NS, int CPT, int MINB>
+cudaError_t launch_scan(attamba_dtype_t dtype, const ScanArgs& a, cudaStream_t s) {
   // about ATTAMBA_SCAN_TOKENS tokens of chunks per block
   int64_t cpb = ((int64_t)ATTAMBA_SCAN_TOKENS * a.n_chunks) / (a.T > 0 ? a.T : 1);
   if (cpb < 1) cpb = 1;
@@ -299,10 +315,17 @@ cudaError_t launch_kv_ssm_scan(attamba_dtype_t dtype, const ScanArgs& a, cudaStr
   if ((a.n_chunks + cpb - 1) / cpb > 65535) return cudaErrorInvalidValue;
   dim3 grid((a.D / CPT + kScanThreads - 1) / kScanThreads, (unsigned)((a.n_chunks + cpb - 1) / cpb), 2);
   if (dtype == ATTAMBA_BF16)
-    kv_ssm_scan_kernel<__nv_bfloat16, CPT, ATTAMBA_SCAN_POLY_PAIRS><<<grid, kScanThreads, 0, s>>>(a, (int32_t)cpb);
+    kv_ssm_scan_kernel<__nv_bfloat16, CPT, NS, NS == 16 ? ATTAMBA_SCAN_POLY_PAIRS : 0, MINB>
+        <<<grid, kScanThreads, 0, s>>>(a, (int32_t)cpb);
   else
-    kv_ssm_scan_kernel<float, CPT, 0><<<grid, kScanThreads, 0, s>>>(a, (int32_t)cpb);
+    kv_ssm_scan_kernel<float, CPT, NS, 0, MINB><<<grid, kScanThreads, 0, s>>>(a, (int32_t)cpb);
   return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_kv_ssm_scan(attamba_dtype_t dtype, const ScanArgs& a, cudaStream_t s) {
+  if (a.N == 32) return launch_scan<32, 1, 3>(dtype, a, s);
+  return launch_scan<16, ATTAMBA_SCAN_CPT, ATTAMBA_SCAN_MINB>(dtype, a, s);
 }
 
 }  // namespace attamba

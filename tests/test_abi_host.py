@@ -55,7 +55,7 @@ def test_invalid_arguments_are_rejected_on_the_host():
     assert lib.attamba_chunk_index(None, 4, 1, 16, 4, 0, -1, 0, ctypes.byref(idx3), None, None) == A.ERR_INVALID_ARG
     # scan: unsupported state size, misaligned pointer
     p = [fake] * 12
-    assert lib.attamba_kv_ssm_scan(1, *p, 4, 16, 64, 32, fake, fake, None, None, None, None) == A.ERR_UNSUPPORTED
+    assert lib.attamba_kv_ssm_scan(1, *p, 4, 16, 64, 24, fake, fake, None, None, None, None) == A.ERR_UNSUPPORTED
     p_bad = [fake + 2] + [fake] * 11
     assert lib.attamba_kv_ssm_scan(1, *p_bad, 4, 16, 64, 16, fake, fake, None, None, None, None) == A.ERR_INVALID_ARG
     # attention: head_dim other than 64

@@ -84,11 +84,11 @@ def test_decode_workload_128_steps():
         assert torch.equal(cache.Kb[:, :, last], cache.Kr[:, :, p % cfg.L])
 
 
-@pytest.mark.parametrize("P,offset,L", [(4, 0, 3), (8, 3, 8), (3, 1, 1)])
-def test_decode_from_empty_cache_equals_test_mask_prefill(P, offset, L):
+@pytest.mark.parametrize("P,offset,L,N", [(4, 0, 3, 16), (8, 3, 8, 16), (3, 1, 1, 16), (8, 3, 8, 32)])
+def test_decode_from_empty_cache_equals_test_mask_prefill(P, offset, L, N):
     """Decoding n tokens one by one from an empty cache reproduces the M_test prefill (GPU vs GPU and vs oracle)."""
-    B, n, H, dh, N = 2, 150, 2, 64, 16
-    cfg = W.shrink(W.LAYER_CONFIGS[2], B=B, n=n, D=H * dh, H=H, P=P, offset=offset, L=L, mode="test")
+    B, n, H, dh = 2, 150, 2, 64
+    cfg = W.shrink(W.LAYER_CONFIGS[2], B=B, n=n, D=H * dh, H=H, P=P, offset=offset, L=L, mode="test", N=N)
     inp = W.make_layer(cfg)
     pf = run_prefill(inp, cfg)
     cap = n // P + 2

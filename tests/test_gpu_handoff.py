@@ -32,12 +32,13 @@ def _empty_cache(B, H, dh, N, P, offset, L, cap):
                    P, offset)
 
 
-@pytest.mark.parametrize("P,offset,L,n0", [(8, 3, 16, 300), (4, 0, 8, 256), (8, 0, 64, 40), (3, 1, 1, 100)])
-def test_cache_from_prefill_matches_oracle_and_continues_the_prefill(P, offset, L, n0):
-    B, H, dh, N, m = 2, 2, 64, 16, 24
+@pytest.mark.parametrize("P,offset,L,n0,N", [(8, 3, 16, 300, 16), (4, 0, 8, 256, 16), (8, 0, 64, 40, 16),
+                                             (3, 1, 1, 100, 16), (8, 3, 16, 300, 32)])
+def test_cache_from_prefill_matches_oracle_and_continues_the_prefill(P, offset, L, n0, N):
+    B, H, dh, m = 2, 2, 64, 24
     n = n0 + m
     D = H * dh
-    cfg = W.shrink(W.LAYER_CONFIGS[2], B=B, n=n, D=D, H=H, P=P, offset=offset, L=L, mode="test")
+    cfg = W.shrink(W.LAYER_CONFIGS[2], B=B, n=n, D=D, H=H, P=P, offset=offset, L=L, mode="test", N=N)
     inp = W.make_layer(cfg)
     pf = run_prefill(inp, cfg)                      # M_test prefill over all n positions (reference rows)
     g = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}

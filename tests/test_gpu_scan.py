@@ -18,10 +18,13 @@ SMALL = [
     W.shrink(W.LAYER_CONFIGS[1], B=1, n=64, D=64, H=1, P=1, offset=0),   # P = 1
     W.shrink(W.LAYER_CONFIGS[1], B=2, n=50, D=64, H=1, P=64, offset=0),  # one chunk per sequence
     W.shrink(W.LAYER_CONFIGS[0], B=2, n=77, D=64, H=1, P=16, offset=5),   # fp32 cyclic
+    W.shrink(W.LAYER_CONFIGS[2], B=2, n=200, D=128, H=2, N=32),           # state size 32 (the pages' default)
+    W.shrink(W.LAYER_CONFIGS[3], B=2, n=150, D=64, H=1, N=32),            # N = 32, variable chunks
+    W.shrink(W.LAYER_CONFIGS[0], B=1, n=96, D=64, H=1, N=32, offset=2),   # fp32, N = 32
 ]
 
 
-@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: f"{c.name}-B{c.B}-n{c.n}-D{c.D}-P{c.P}")
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: f"{c.name}-B{c.B}-n{c.n}-D{c.D}-P{c.P}-N{c.N}")
 def test_scan_small(cfg):
     inp = W.make_layer(cfg)
     pf = run_prefill(inp, cfg)
