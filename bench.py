@@ -281,6 +281,74 @@ def decode_bench(dev, reps=3):
             "gpu_launches_per_step": 3}
 
 
+def next_rows_bench(cfg, g, inp, pf, nch, dev, flush, scan_exps, reps=10):
+    """The rows built after the hot path, timed on the bench workload's shapes (L2 flushed before each
+    launch, median of CUDA-event times on the launching stream): the kept-projection scan (one input per
+    SSM), the scan at the pages' state size N = 32, and the prefill -> decode cache handoff."""
+    import math
+    from ssm_compressed_chunked_b200 import attamba as A
+
+    stream = torch.cuda.current_stream(dev)
+    exp_peak = 16 * 148 * 1.965e9
+    hbm = peaks()[0]
+
+    def timed(fn):
+        ts = []
+        for _ in range(reps + 2):
+            flush.fill_(3)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return float(np.median(ts[2:]))  # ms
+
+    T, D, H, dh = cfg.B * cfg.n, cfg.D, cfg.H, cfg.dh
+    flat = lambda t: t.reshape(T, -1)
+    K2, V2 = torch.empty_like(pf.K), torch.empty_like(pf.V)
+    Kc2, Vc2 = torch.empty_like(pf.Kc), torch.empty_like(pf.Vc)
+    rows = {}
+    # f3: the values SSM reads a second [T, D] input (q's memory stands in for x W_V)
+    ms = timed(lambda: A.kv_ssm_scan_u(flat(g["x"]), flat(g["q"]), flat(g["dt_k"]), flat(g["dt_v"]), g["bias_k"],
+                                       g["bias_v"], g["A_k"], g["A_v"], flat(g["B_k"]), flat(g["C_k"]), flat(g["B_v"]),
+                                       flat(g["C_v"]), pf.index.cu, nch, K2, V2, Kc2, Vc2, pf.status))
+    rows["f3_scan_kept_projection"] = {"us": ms * 1e3, "Gexp_s": scan_exps / (ms * 1e-3) / 1e9,
+                                       "frac_of_exp_unit": scan_exps / (ms * 1e-3) / exp_peak}
+    # f4: N = 32, B / C ~ N(0, 1) and A = -exp(U(log 1, log 16)) like the workload's, drawn here
+    gen = torch.Generator().manual_seed(32)
+    N2 = 32
+    bc = [torch.randn(T, N2, generator=gen).to(torch.bfloat16).to(dev) for _ in range(4)]
+    A32 = [(-torch.exp(torch.rand(D, N2, generator=gen) * math.log(16.0))).to(dev) for _ in range(2)]
+    ms = timed(lambda: A.kv_ssm_scan(flat(g["x"]), flat(g["dt_k"]), flat(g["dt_v"]), g["bias_k"], g["bias_v"],
+                                     A32[0], A32[1], bc[0], bc[1], bc[2], bc[3], pf.index.cu, nch, K2, V2, Kc2, Vc2,
+                                     pf.status))
+    exps32 = 2.0 * T * D * N2
+    rows["f4_scan_N32"] = {"us": ms * 1e3, "Gexp_s": exps32 / (ms * 1e-3) / 1e9,
+                           "frac_of_exp_unit": exps32 / (ms * 1e-3) / exp_peak}
+    # f2: the cache a prefill of the whole sequence leaves (uniform chunks; L leading tokens)
+    L = max(1, cfg.L)
+    cap = cfg.n // cfg.P + 2
+    bf = torch.bfloat16
+    cache = A.Cache(torch.zeros(2, cfg.B, cfg.N, D, device=dev), torch.zeros(cfg.B, H, cap, dh, dtype=bf, device=dev),
+                    torch.zeros(cfg.B, H, cap, dh, dtype=bf, device=dev),
+                    torch.zeros(cfg.B, cap, dtype=torch.int32, device=dev),
+                    torch.zeros(cfg.B, H, L, dh, dtype=bf, device=dev), torch.zeros(cfg.B, H, L, dh, dtype=bf, device=dev),
+                    torch.zeros(cfg.B, dtype=torch.int32, device=dev), torch.zeros(cfg.B, dtype=torch.int32, device=dev),
+                    cfg.P, cfg.offset)
+    Kv, Vv = pf.K.view(cfg.B, cfg.n, H, dh), pf.V.view(cfg.B, cfg.n, H, dh)
+    ms = timed(lambda: A.cache_from_prefill(cache, Kv, Vv, flat(g["x"]), flat(g["dt_k"]), flat(g["dt_v"]), g["bias_k"],
+                                            g["bias_v"], g["A_k"], g["A_v"], flat(g["B_k"]), flat(g["C_k"]),
+                                            flat(g["B_v"]), flat(g["C_v"]), cfg.n, pf.status))
+    nb = int(cache.nb[0].item())
+    hbytes = cfg.B * ((nb + min(L, cfg.n)) * 2 * D * 2 * 2 + 2 * cfg.N * D * 4 + cfg.P * (3 * D * 2 + 4 * cfg.N * 2))
+    rows["f2_cache_from_prefill"] = {"us": ms * 1e3, "bytes": hbytes, "GB_s": hbytes / (ms * 1e-3) / 1e9,
+                                     "frac_of_hbm": hbytes / (ms * 1e-3) / 1e9 / hbm,
+                                     "note": "launch-bound at this size (a few MB)"}
+    assert pf.status.item() == 0, f"device status {pf.status.item()}"
+    return rows
+
+
 # ------------------------------------------------------------------ CUDA path
 def run_ours(args, ws, rank, local):
     from ssm_compressed_chunked_b200 import attamba as A, layer
@@ -424,11 +492,13 @@ def run_ours(args, ws, rank, local):
         "attn_tensor": {"achieved_TFLOP_s": attn_flops / (mean[2] * 1e-3) / 1e12,
                         "frac_of_burst": attn_flops / (mean[2] * 1e-3) / 1e12 / tf_burst},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 3 * args.steps,
         "clocks": clocks,
     }
     if ws == 1 and not args.no_decode:
         out["decode"] = decode_bench(dev)
+    if ws == 1 and not args.no_next_rows:
+        out["next_rows"] = next_rows_bench(cfg, g, inp, pf, nch, dev, flush, scan_exps)
     if ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline()
     print(json.dumps(out), flush=True)
@@ -442,6 +512,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-row measurement")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip timing the rows built after the hot path (kept projections, N = 32, handoff)")
     ap.add_argument("--min-warmup-ms", type=float, default=500.0,
                     help="keep warming up at least this long so clocks have ramped (0 under a profiler)")
     args = ap.parse_args()

@@ -198,7 +198,7 @@ __device__ __forceinline__ void scan_token(ScanState<CPT, NS>& st, const float* 
   }
 }
 
-template <typename T, int CPT, int NS, int POLY_PAIRS, int MINB>
+template <typename T, int CPT, int NS, int POLY_PAIRS, int MINB, bool SPLIT_X>
 __global__ void __launch_bounds__(kScanThreads, MINB) kv_ssm_scan_kernel(ScanArgs p, int32_t chunks_per_block) {
   using V = Vec<T, CPT>;
   constexpr int kNS = NS;
@@ -215,7 +215,9 @@ __global__ void __launch_bounds__(kScanThreads, MINB) kv_ssm_scan_kernel(ScanArg
   const int32_t c_end = min(c_begin + chunks_per_block, p.n_chunks);
   for (int i = threadIdx.x; i <= c_end - c_begin; i += kScanThreads) sCu[i] = p.cu[c_begin + i];
 
-  const T* __restrict__ x = static_cast<const T*>(p.x[s]) + d0;
+  // one input for both SSMs unless SPLIT_X (kept projections): a base chosen per grid z
+  // measured 7% slower on the shared-input workload, so the shared case reads x[0] directly
+  const T* __restrict__ x = static_cast<const T*>(SPLIT_X ? p.x[s] : p.x[0]) + d0;
   const T* __restrict__ dt = static_cast<const T*>(p.dt[s]) + d0;
   const T* __restrict__ Bm = static_cast<const T*>(p.Bm[s]);
   const T* __restrict__ Cm = static_cast<const T*>(p.Cm[s]);
@@ -306,7 +308,7 @@ __global__ void __launch_bounds__(kScanThreads, MINB) kv_ssm_scan_kernel(ScanArg
 
 namespace {
 // N = 16: two channels per thread; N = 32: one (the state and A of two channels would not fit)
-template <int NS, int CPT, int MINB>
+template <int NS, int CPT, int MINB, bool SPLIT_X>
 cudaError_t launch_scan(attamba_dtype_t dtype, const ScanArgs& a, cudaStream_t s) {
   // about ATTAMBA_SCAN_TOKENS tokens of chunks per block
   int64_t cpb = ((int64_t)ATTAMBA_SCAN_TOKENS * a.n_chunks) / (a.T > 0 ? a.T : 1);
@@ -315,17 +317,19 @@ cudaError_t launch_scan(attamba_dtype_t dtype, const ScanArgs& a, cudaStream_t s
   if ((a.n_chunks + cpb - 1) / cpb > 65535) return cudaErrorInvalidValue;
   dim3 grid((a.D / CPT + kScanThreads - 1) / kScanThreads, (unsigned)((a.n_chunks + cpb - 1) / cpb), 2);
   if (dtype == ATTAMBA_BF16)
-    kv_ssm_scan_kernel<__nv_bfloat16, CPT, NS, NS == 16 ? ATTAMBA_SCAN_POLY_PAIRS : 0, MINB>
+    kv_ssm_scan_kernel<__nv_bfloat16, CPT, NS, NS == 16 ? ATTAMBA_SCAN_POLY_PAIRS : 0, MINB, SPLIT_X>
         <<<grid, kScanThreads, 0, s>>>(a, (int32_t)cpb);
   else
-    kv_ssm_scan_kernel<float, CPT, NS, 0, MINB><<<grid, kScanThreads, 0, s>>>(a, (int32_t)cpb);
+    kv_ssm_scan_kernel<float, CPT, NS, 0, MINB, SPLIT_X><<<grid, kScanThreads, 0, s>>>(a, (int32_t)cpb);
   return cudaGetLastError();
 }
 }  // namespace
 
 cudaError_t launch_kv_ssm_scan(attamba_dtype_t dtype, const ScanArgs& a, cudaStream_t s) {
-  if (a.N == 32) return launch_scan<32, 1, 3>(dtype, a, s);
-  return launch_scan<16, ATTAMBA_SCAN_CPT, ATTAMBA_SCAN_MINB>(dtype, a, s);
+  const bool split = a.x[0] != a.x[1];
+  if (a.N == 32) return split ? launch_scan<32, 1, 3, true>(dtype, a, s) : launch_scan<32, 1, 3, false>(dtype, a, s);
+  return split ? launch_scan<16, ATTAMBA_SCAN_CPT, ATTAMBA_SCAN_MINB, true>(dtype, a, s)
+               : launch_scan<16, ATTAMBA_SCAN_CPT, ATTAMBA_SCAN_MINB, false>(dtype, a, s);
 }
 
 }  // namespace attamba
