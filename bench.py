@@ -283,8 +283,8 @@ def decode_bench(dev, reps=3):
 
 def next_rows_bench(cfg, g, inp, pf, nch, dev, flush, scan_exps, reps=10):
     """The rows built after the hot path, timed on the bench workload's shapes (L2 flushed before each
-    launch, median of CUDA-event times on the launching stream): the kept-projection scan (one input per
-    SSM), the scan at the pages' state size N = 32, and the prefill -> decode cache handoff."""
+    launch, median of CUDA-event times on the launching stream): the projection GEMMs, the kept-projection
+    scan (one input per SSM), the scan at the pages' state size N = 32, and the prefill -> decode handoff."""
     import math
     from ssm_compressed_chunked_b200 import attamba as A
 
@@ -345,6 +345,25 @@ def next_rows_bench(cfg, g, inp, pf, nch, dev, flush, scan_exps, reps=10):
     rows["f2_cache_from_prefill"] = {"us": ms * 1e3, "bytes": hbytes, "GB_s": hbytes / (ms * 1e-3) / 1e9,
                                      "frac_of_hbm": hbytes / (ms * 1e-3) / 1e9 / hbm,
                                      "note": "launch-bound at this size (a few MB)"}
+    # f1: the layer's seven input projections as one GEMM (q | dt_K | dt_V | B_K | C_K | B_V | C_V, random-init
+    # weights of the workload's shapes), and the output projection
+    tf_burst = peaks()[1]
+    widths = [H * dh, D, D, cfg.N, cfg.N, cfg.N, cfg.N]
+    W_in = (torch.randn(sum(widths), D, generator=gen) / math.sqrt(D)).to(bf).to(dev)
+    outs, c = [], 0
+    for w in widths:
+        outs.append((torch.empty(T, w, dtype=bf, device=dev), c))
+        c += w
+    ms_in = timed(lambda: A.proj_gemm(flat(g["x"]), W_in, outs, pf.status))
+    W_O = (torch.randn(D, H * dh, generator=gen) / math.sqrt(D)).to(bf).to(dev)
+    y = torch.empty(T, D, dtype=bf, device=dev)
+    ms_o = timed(lambda: A.proj_gemm(pf.O.view(T, H * dh), W_O, [(y, 0)], pf.status))
+    fl_in, fl_o = 2.0 * T * sum(widths) * D, 2.0 * T * D * H * dh
+    rows["f1_projection_gemm"] = {
+        "inputs": {"us": ms_in * 1e3, "TFLOP_s": fl_in / (ms_in * 1e-3) / 1e12,
+                   "frac_of_bf16_burst": fl_in / (ms_in * 1e-3) / 1e12 / tf_burst},
+        "output": {"us": ms_o * 1e3, "TFLOP_s": fl_o / (ms_o * 1e-3) / 1e12,
+                   "frac_of_bf16_burst": fl_o / (ms_o * 1e-3) / 1e12 / tf_burst}}
     assert pf.status.item() == 0, f"device status {pf.status.item()}"
     return rows
 

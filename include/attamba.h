@@ -109,6 +109,29 @@ attamba_status_t attamba_chunk_index(const int32_t* cu_in, int32_t n_chunks, int
                                      const attamba_index_t* out, int32_t* d_status,
                                      attamba_stream_t stream);
 
+/* One output segment of attamba_proj_gemm: columns [col0, col0 + width) of Y,
+ * written to ptr as a row-major [M, width] bf16 array. */
+typedef struct {
+  void* ptr;
+  int32_t col0;
+  int32_t width;
+} attamba_proj_seg_t;
+
+/* attamba_proj_gemm -- the layer's projections as one tensor-core GEMM, Y = X W^T.
+ * [pith, core] the SSMs replace W_K and W_V, the query and output projections stay;
+ * [pith, params] the selective SSM's step and B, C are projections of the input.
+ * The seven input projections (W_Q, W_dK, W_dV, W_BK, W_CK, W_BV, W_CV stacked along
+ * their output features) are one call whose segments are q, dt_k, dt_v, B_k, C_k,
+ * B_v, C_v; the output projection W_O is another with one segment.
+ *   X      [M, K] bf16 row-major;  W  [Nout, K] bf16 row-major (output x input features).
+ *   segs   nseg (1..8) segments, sorted by col0, not overlapping, col0 and width
+ *          multiples of 8, col0 + width <= Nout; columns no segment names are not written.
+ *   K      a multiple of 64.  fp32 accumulation, bf16 rounding of Y.
+ * X, W and every segment pointer 16-byte aligned.  bf16 only. */
+attamba_status_t attamba_proj_gemm(attamba_dtype_t dtype, const void* X, const void* W, int64_t M, int32_t Nout,
+                                   int32_t K, const attamba_proj_seg_t* segs, int32_t nseg, int32_t* d_status,
+                                   attamba_stream_t stream);
+
 /* attamba_kv_ssm_scan -- both KV-SSMs over the layer input, state reset at chunk starts.
  * [pith, core] K = SSM_K(X), V = SSM_V(X); [pith, params] Mamba selective SSM (Eq. 3);
  * [pith, carries] one state per chunk of P tokens.  Per token t, channel d, SSM s:

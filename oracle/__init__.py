@@ -18,6 +18,7 @@ mask       M_train / M_test / leading-token masks, dense from the definition,
            and the canonical compact key index derived from the same definition
 attention  dense masked softmax attention (whole rows and sampled rows)
 decode     one-token-at-a-time decode over the boundary-state cache
+projection the layer's linear projections (kept W_Q, W_O; the SSMs' Delta, B, C)
 scalar     literal scalar loops for tiny shapes (brute-force cross-check)
 
 Every function states which passage it follows.  Where the pages are silent the
@@ -26,4 +27,4 @@ design notes.  Every function is pinned by ``tests/test_oracle_*.py`` against
 closed forms, invariants, brute force and the page's own worked count.
 """
 
-from . import chunks, ssm, mask, attention, decode, scalar  # noqa: F401
+from . import chunks, ssm, mask, attention, decode, projection, scalar  # noqa: F401

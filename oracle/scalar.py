@@ -67,3 +67,16 @@ def attention(q, k, v, allowed, scale):
         z = sum(w)
         out.append([sum(w[a] * v[keys[a]][c] for a in range(len(keys))) / z for c in range(dh)])
     return out
+
+
+def project(x, W):
+    """y[m, o] = sum_k x[m, k] W[o, k], one number at a time (brute force for tiny shapes)."""
+    M, K = len(x), len(x[0])
+    out = [[0.0] * len(W) for _ in range(M)]
+    for m in range(M):
+        for o in range(len(W)):
+            acc = 0.0
+            for k in range(K):
+                acc += float(x[m][k]) * float(W[o][k])
+            out[m][o] = acc
+    return out

@@ -26,7 +26,7 @@ EXPORTS = ("attamba_version", "attamba_status_string", "attamba_last_error",
            "attamba_uniform_chunk_count", "attamba_chunk_index", "attamba_kv_ssm_scan",
            "attamba_chunk_attn_fwd", "attamba_decode_workspace_size", "attamba_decode_step",
            "attamba_decode_step_noalloc", "attamba_cache_from_prefill",
-           "attamba_kv_ssm_scan_u")
+           "attamba_kv_ssm_scan_u", "attamba_proj_gemm")
 
 
 class AttambaError(RuntimeError):
@@ -37,6 +37,10 @@ class IndexT(ctypes.Structure):
     _fields_ = [("cu", ctypes.c_void_p), ("bpos", ctypes.c_void_p), ("bptr", ctypes.c_void_p),
                 ("ls", ctypes.c_void_p), ("nbb", ctypes.c_void_p),
                 ("n_chunks", ctypes.c_int32), ("B", ctypes.c_int32), ("n", ctypes.c_int32)]
+
+
+class ProjSegT(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("col0", ctypes.c_int32), ("width", ctypes.c_int32)]
 
 
 class CacheT(ctypes.Structure):
@@ -69,6 +73,8 @@ def load():
                                       ctypes.POINTER(IndexT), vp, vp]
     L.attamba_kv_ssm_scan.restype = ctypes.c_int
     L.attamba_kv_ssm_scan.argtypes = [ctypes.c_int] + [vp] * 12 + [i32, i64, i32, i32] + [vp] * 4 + [vp, vp]
+    L.attamba_proj_gemm.restype = ctypes.c_int
+    L.attamba_proj_gemm.argtypes = [ctypes.c_int, vp, vp, i64, i32, i32, ctypes.POINTER(ProjSegT), i32, vp, vp]
     L.attamba_kv_ssm_scan_u.restype = ctypes.c_int
     L.attamba_kv_ssm_scan_u.argtypes = [ctypes.c_int] + [vp] * 13 + [i32, i64, i32, i32] + [vp] * 4 + [vp, vp]
     L.attamba_chunk_attn_fwd.restype = ctypes.c_int
@@ -267,3 +273,21 @@ def cache_from_prefill(cache, K, V, x, dt_k, dt_v, bias_k, bias_v, A_k, A_v, B_k
         _ptr(B_v, dt, "B_v"), _ptr(C_v, dt, "C_v"), int(n0),
         _ptr(status, torch.int32, "status", allow_none=True), _stream(stream))
     _check(st, "attamba_cache_from_prefill")
+
+
+def proj_gemm(X, W, outs, status=None, stream=None):
+    """attamba_proj_gemm: Y = X W^T (bf16, fp32 accumulation) with Y's columns split into `outs`, a list of
+    (tensor [M, width] bf16, first column) pairs in column order.  X: [M, K]; W: [Nout, K]."""
+    bf = torch.bfloat16
+    M, K = X.shape
+    Nout = W.shape[0]
+    if W.shape[1] != K:
+        raise AttambaError("W must be [Nout, K] with X's K")
+    segs = (ProjSegT * len(outs))()
+    for k, (t, c0) in enumerate(outs):
+        if t.dim() != 2 or t.shape[0] != M:
+            raise AttambaError("each output must be [M, width]")
+        segs[k] = ProjSegT(_ptr(t, bf, "out"), int(c0), int(t.shape[1]))
+    st = load().attamba_proj_gemm(BF16, _ptr(X, bf, "X"), _ptr(W, bf, "W"), M, Nout, K, segs, len(outs),
+                                  _ptr(status, torch.int32, "status", allow_none=True), _stream(stream))
+    _check(st, "attamba_proj_gemm")

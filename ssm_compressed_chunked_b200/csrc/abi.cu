@@ -121,6 +121,33 @@ attamba_status_t attamba_kv_ssm_scan_u(attamba_dtype_t dtype, const void* u_k, c
                     N, K, V, Kc, Vc, d_status, reinterpret_cast<cudaStream_t>(stream), "attamba_kv_ssm_scan_u");
 }
 
+attamba_status_t attamba_proj_gemm(attamba_dtype_t dtype, const void* X, const void* W, int64_t M, int32_t Nout,
+                                   int32_t K, const attamba_proj_seg_t* segs, int32_t nseg, int32_t* d_status,
+                                   attamba_stream_t stream) {
+  if (dtype != ATTAMBA_BF16) return ATTAMBA_ERR_UNSUPPORTED;
+  if (M < 1 || Nout < 1 || K < 64 || K % 64 != 0 || !segs || nseg < 1 || nseg > attamba::kMaxProjSegs)
+    return ATTAMBA_ERR_INVALID_ARG;
+  if (M >= ((int64_t)1 << 31) || M * (int64_t)K >= ((int64_t)1 << 40) || M * (int64_t)Nout >= ((int64_t)1 << 40))
+    return ATTAMBA_ERR_INVALID_ARG;
+  if (!X || !W || !aligned16(X) || !aligned16(W)) return ATTAMBA_ERR_INVALID_ARG;
+  attamba::ProjArgs a{};
+  a.X = X; a.W = W; a.M = M; a.Nout = Nout; a.K = K; a.nseg = nseg; a.status = d_status;
+  int32_t end = 0;
+  for (int s = 0; s < nseg; ++s) {
+    const attamba_proj_seg_t& g = segs[s];
+    if (!g.ptr || !aligned16(g.ptr) || g.col0 < end || g.width < 8 || g.col0 % 8 != 0 || g.width % 8 != 0 ||
+        (int64_t)g.col0 + g.width > Nout)
+      return ATTAMBA_ERR_INVALID_ARG;
+    a.seg_ptr[s] = g.ptr;
+    a.seg_col0[s] = g.col0;
+    a.seg_width[s] = g.width;
+    end = g.col0 + g.width;
+  }
+  cudaError_t e = attamba::launch_proj_gemm(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) return ATTAMBA_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? ATTAMBA_OK : cuda_fail(e, "attamba_proj_gemm");
+}
+
 attamba_status_t attamba_chunk_attn_fwd(attamba_dtype_t dtype, const void* q, const void* K,
                                         const void* V, const void* Kc, const void* Vc,
                                         const attamba_index_t* idx, int32_t H, int32_t dh,

@@ -50,6 +50,22 @@
 
 namespace attamba {
 
+// the driver's tensor-map encoder, resolved once at run time (the library links no driver API)
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
 namespace {
 constexpr int kBM = 128;                                    // queries per work item (TMEM lanes)
 constexpr int kBN = 64;                                     // keys per tile
@@ -600,24 +616,9 @@ __global__ void __launch_bounds__(128) chunk_attn_f32_kernel(AttnArgs a) {
 }
 
 // ---------------------------------------------------------------- tensor maps
-PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
 // [rows, H, 64] bf16 viewed as a 3-D tensor; box = 64 x 1 x box_rows with the 128-byte swizzle
 bool encode_rows_map(CUtensorMap* m, const void* base, int64_t rows, int H, int box_rows) {
-  auto enc = get_encoder();
+  auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)kDH, (cuuint64_t)H, (cuuint64_t)rows};
   cuuint64_t strides[2] = {(cuuint64_t)kDH * 2, (cuuint64_t)H * kDH * 2};

@@ -1,12 +1,17 @@
 // Internal launchers behind the C ABI (abi.cu validates, these launch).
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include "attamba.h"
 
 namespace attamba {
+
+// cuTensorMapEncodeTiled from the driver (null when unavailable)
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 cudaError_t launch_chunk_index(const int32_t* cu_in, int32_t n_chunks, int32_t B, int32_t n,
                                int32_t P, int32_t offset, int32_t L, int mode,
@@ -70,6 +75,21 @@ size_t decode_workspace_bytes(const attamba_cache_t& c);
 size_t decode_noalloc_scratch_bytes();
 cudaError_t decode_noalloc_scratch(float** out);
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s);
+
+constexpr int kMaxProjSegs = 8;
+struct ProjArgs {
+  const void* X;   // [M, K]
+  const void* W;   // [Nout, K]
+  int64_t M;
+  int32_t Nout;
+  int32_t K;
+  int32_t nseg;
+  void* seg_ptr[kMaxProjSegs];     // segment s: columns [col0, col0 + width) -> [M, width]
+  int32_t seg_col0[kMaxProjSegs];
+  int32_t seg_width[kMaxProjSegs];
+  int32_t* status;
+};
+cudaError_t launch_proj_gemm(const ProjArgs& a, cudaStream_t s);
 
 struct HandoffArgs {
   attamba_cache_t c;
