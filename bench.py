@@ -363,7 +363,8 @@ def next_rows_bench(cfg, g, inp, pf, nch, dev, flush, scan_exps, reps=10):
         "inputs": {"us": ms_in * 1e3, "TFLOP_s": fl_in / (ms_in * 1e-3) / 1e12,
                    "frac_of_bf16_burst": fl_in / (ms_in * 1e-3) / 1e12 / tf_burst},
         "output": {"us": ms_o * 1e3, "TFLOP_s": fl_o / (ms_o * 1e-3) / 1e12,
-                   "frac_of_bf16_burst": fl_o / (ms_o * 1e-3) / 1e12 / tf_burst}}
+                   "frac_of_bf16_burst": fl_o / (ms_o * 1e-3) / 1e12 / tf_burst},
+        "traffic_inputs": ncu_traffic("proj_gemm_kernel")}
     assert pf.status.item() == 0, f"device status {pf.status.item()}"
     return rows
 

@@ -15,7 +15,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libattamba.so")
-SOURCES = ["abi.cu", "chunk_index.cu", "kv_ssm_scan.cu", "chunk_attn.cu", "decode.cu", "handoff.cu", "proj_gemm.cu"]
+SOURCES = ["abi.cu", "chunk_index.cu", "kv_ssm_scan.cu", "chunk_attn.cu", "decode.cu", "handoff.cu", "proj_gemm.cu", "device.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "-shared", "-cudart", "static", "-I", INCLUDE, "-I", CSRC]

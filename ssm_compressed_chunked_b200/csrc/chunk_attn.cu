@@ -52,17 +52,16 @@ namespace attamba {
 
 // the driver's tensor-map encoder, resolved once at run time (the library links no driver API)
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  // resolved once (thread-safe static initialisation)
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+  }();
   return fn;
 }
 
@@ -639,20 +638,9 @@ cudaError_t launch_chunk_attn_bf16(const AttnArgs& a, cudaStream_t s) {
       !encode_rows_map(&tv, a.V, T, a.H, kBN) || !encode_rows_map(&tkc, a.Kc, a.n_chunks, a.H, kBN) ||
       !encode_rows_map(&tvc, a.Vc, a.n_chunks, a.H, kBN))
     return cudaErrorNotSupported;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(chunk_attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
+  cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(chunk_attn_bf16_kernel), (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int sms = device_sm_count();
   // persistent: two CTAs per SM, each walking the work items (sequence, head, 128 queries) round
   // robin; more CTAs only when a CTA would hold more items than its table
   const int64_t items = (int64_t)((a.n + kBM - 1) / kBM) * a.B * a.H;

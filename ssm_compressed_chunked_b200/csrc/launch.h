@@ -12,6 +12,10 @@ namespace attamba {
 
 // cuTensorMapEncodeTiled from the driver (null when unavailable)
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+// SM count of the current device (cached per device)
+int device_sm_count();
+// raise `kernel`'s dynamic shared-memory limit on the current device, once per device
+cudaError_t raise_smem_limit(const void* kernel, int bytes);
 
 cudaError_t launch_chunk_index(const int32_t* cu_in, int32_t n_chunks, int32_t B, int32_t n,
                                int32_t P, int32_t offset, int32_t L, int mode,

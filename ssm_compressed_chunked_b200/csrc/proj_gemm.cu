@@ -221,19 +221,9 @@ bool encode_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int
 cudaError_t launch_proj_gemm(const ProjArgs& a, cudaStream_t s) {
   CUtensorMap tx, tw;
   if (!encode_2d(&tx, a.X, a.M, a.K, kBM) || !encode_2d(&tw, a.W, a.Nout, a.K, kBN)) return cudaErrorNotSupported;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(proj_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
+  cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(proj_gemm_kernel), (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int sms = device_sm_count();
   const int64_t tiles = ((a.M + kBM - 1) / kBM) * ((a.Nout + kBN - 1) / kBN);
   const int grid = (int)(tiles < sms ? tiles : sms);
   proj_gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(tx, tw, a);
