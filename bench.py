@@ -278,7 +278,7 @@ def decode_bench(dev, reps=3):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                          "peak_source": f"{src} HBM copy", "traffic": ncu_traffic("decode_attn_kernel"),
                          "traffic_kernel": "decode_attn_kernel"},
-            "gpu_launches_per_step": 3}
+            "gpu_launches_per_step": 2}
 
 
 def next_rows_bench(cfg, g, inp, pf, nch, dev, flush, scan_exps, reps=10):

@@ -7,15 +7,15 @@
 // tokens (Eq. 8); Referee Report, comment on Eq. (7) -- the current chunk is
 // reached only through the leading tokens.
 //
-// Three stream-ordered launches, no inter-CTA waiting:
-//   decode_ssm_kernel     per (channel, sequence, SSM): reset at a chunk start,
-//                         one state update (state [2,B,N,D] read and written
-//                         coalesced), k_t / v_t into ring slot t mod L and, at a
-//                         chunk end, into the boundary list
-//   decode_attn_kernel    per (split, head, sequence): streams its share of the
+// Two stream-ordered launches, no inter-CTA waiting:
+//   decode_attn_kernel    per (split, head, sequence): the last split first runs the
+//                         SSM step of the head's channels (reset at a chunk start,
+//                         state [2,B,N,D] read and written coalesced, k_t / v_t into
+//                         ring slot t mod L and, at a chunk end, into the boundary
+//                         list); every split then streams its share of the
 //                         (boundaries below the window) + (window) keys with
-//                         16-byte loads, 8 lanes per key row, fp32 online softmax;
-//                         writes (max, sum, unnormalised output) to the workspace
+//                         16-byte loads, 8 lanes per key row, fp32 online softmax,
+//                         and writes (max, sum, unnormalised output) to the workspace
 //   decode_combine_kernel per (sequence, head): merges the splits, writes o_t,
 //                         and advances pos / nb
 // The step is bound by streaming the cached K/V from HBM.
@@ -49,13 +49,13 @@ __device__ __forceinline__ bool chunk_ends_at(int t, int P, int o) {
   return (t + 1 >= o) && ((t + 1 - o) % P == 0);
 }
 
+// One SSM step of channel d of sequence b for SSM s: reset at a chunk start, state
+// [2,B,N,D] read and written coalesced, k_t / v_t into ring slot t mod L and, at a
+// chunk end, into the boundary list.
 template <int kNS>
-__global__ void __launch_bounds__(128) decode_ssm_kernel(DecodeArgs a) {
+__device__ __forceinline__ void ssm_step(const DecodeArgs& a, int s, int b, int d) {
   const attamba_cache_t& c = a.c;
   const int D = c.H * c.dh;
-  const int s = blockIdx.z, b = blockIdx.y;
-  const int d = blockIdx.x * blockDim.x + threadIdx.x;
-  if (d >= D) return;
   const int o = ((c.offset % c.P) + c.P) % c.P;
   const int t = a.c.pos[b];
   const bool start = chunk_starts_at(t, c.P, o);
@@ -107,10 +107,19 @@ __device__ __forceinline__ void bf16x8_to_f(const uint4& u, float (&f)[8]) {
   }
 }
 
+template <int kNS>
 __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(DecodeArgs a) {
   const attamba_cache_t& c = a.c;
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // The last split of (b, h) holds the newest key (position t): it first runs the SSM step of
+  // the head's 64 channels for both SSMs (one per thread), which writes k_t, v_t into the ring.
+  // No other block reads that slot (it held position t - L, now outside the window), and the
+  // boundary appended at a chunk end lies inside the window, so no other split reads it either.
+  if (split == a.splits - 1) {
+    ssm_step<kNS>(a, threadIdx.x >> 6, b, h * kDH + (threadIdx.x & 63));
+    __syncthreads();
+  }
   const int g = lane >> 3;          // key group within the warp
   const int e8 = (lane & 7) * 8;    // head-dim slice of this lane
   const int L = c.L, cap = c.cap;
@@ -155,17 +164,16 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(DecodeArgs a)
     for (int u = 0; u < kUnroll; ++u) {
       const int k = kk + u * 16 + g;
       if (k < ke) {
-        const __nv_bfloat16 *kp, *vp;
         if (k < nbb) {
-          kp = Kb + (size_t)k * kDH;
-          vp = Vb + (size_t)k * kDH;
+          kr[u] = __ldg(reinterpret_cast<const uint4*>(Kb + (size_t)k * kDH));
+          vr[u] = __ldg(reinterpret_cast<const uint4*>(Vb + (size_t)k * kDH));
         } else {
+          // the ring is written during the step (slot of t): read it through L2, not the
+          // read-only path
           const int slot = (lo + (k - nbb)) % L;
-          kp = Kr + (size_t)slot * kDH;
-          vp = Vr + (size_t)slot * kDH;
+          kr[u] = __ldcg(reinterpret_cast<const uint4*>(Kr + (size_t)slot * kDH));
+          vr[u] = __ldcg(reinterpret_cast<const uint4*>(Vr + (size_t)slot * kDH));
         }
-        kr[u] = __ldg(reinterpret_cast<const uint4*>(kp));
-        vr[u] = __ldg(reinterpret_cast<const uint4*>(vp));
       } else {
         kr[u] = make_uint4(0, 0, 0, 0);
         vr[u] = make_uint4(0, 0, 0, 0);
@@ -328,12 +336,10 @@ size_t decode_workspace_bytes(const attamba_cache_t& c) {
 }
 
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s) {
-  const int D = a.c.H * a.c.dh;
   if (a.c.N == 32)
-    decode_ssm_kernel<32><<<dim3((D + 127) / 128, a.c.B, 2), 128, 0, s>>>(a);
+    decode_attn_kernel<32><<<dim3(a.splits, a.c.H, a.c.B), kAttnThreads, 0, s>>>(a);
   else
-    decode_ssm_kernel<16><<<dim3((D + 127) / 128, a.c.B, 2), 128, 0, s>>>(a);
-  decode_attn_kernel<<<dim3(a.splits, a.c.H, a.c.B), kAttnThreads, 0, s>>>(a);
+    decode_attn_kernel<16><<<dim3(a.splits, a.c.H, a.c.B), kAttnThreads, 0, s>>>(a);
   decode_combine_kernel<<<a.c.B * a.c.H, kDH, 0, s>>>(a);
   return cudaGetLastError();
 }
