@@ -13,7 +13,7 @@
 // tiles (64 keys each) are first the chunk-end tiles 0..nbb(last query), then
 // the local band [ls(first query), last query]; both are plain TMA boxes.
 //   warp 4     TMA producer: Q of each item (two buffers), then K/V tiles into
-//              a 3-stage ring
+//              a 4-stage ring; it also stores each finished O tile
 //   warp 5     one thread issues tcgen05.mma: S = Q K^T (M128 N64 K64, both
 //              operands in shared memory) into TMEM, then O += P V (M128 N64
 //              K64, P read from TMEM, V from shared memory)
@@ -30,8 +30,13 @@
 // P uses a reference max that is raised (and O, l rescaled in TMEM) only when
 // a row's max grows by more than 2^8, so P <= 2^8 and the rescale is rare; the
 // final O / l is exact whatever reference was used.  A full 128-row tile of O
-// leaves through a shared-memory staging tile and one TMA store; a partial
-// tile (the end of a sequence) is written row by row.
+// is staged (128-byte swizzle) in its item's own Q buffer, whose last reader,
+// the item's last QK, has finished by then, and leaves with one TMA store; the
+// producer issues the store and refills the buffer with the Q of the item two
+// ahead only after the store has read it.  A partial tile (the end of a
+// sequence) is written row by row.  At an item boundary the previous item's
+// last PV is issued before the next item's first QK, so the epilogue does not
+// wait for the next item's loads.
 //
 // Measured limits (B200, bench workload): the exponentials of a 64-column
 // tile cost 512 cycles of the multi-function unit per warp, so two CTAs per SM
@@ -70,7 +75,7 @@ constexpr int kBM = 128;                                    // queries per work 
 constexpr int kBN = 64;                                     // keys per tile
 constexpr int kDH = 64;
 #ifndef ATTAMBA_ATTN_STAGES
-#define ATTAMBA_ATTN_STAGES 3
+#define ATTAMBA_ATTN_STAGES 4
 #endif
 #ifndef ATTAMBA_ATTN_CTAS_PER_SM
 #define ATTAMBA_ATTN_CTAS_PER_SM 2
@@ -84,8 +89,7 @@ constexpr uint32_t kKVBytes = kBN * kDH * 2;                // 8 KB: 64 rows x 1
 constexpr uint32_t kQOff = 0;                               // two Q tiles
 constexpr uint32_t kKOff = kQOff + 2 * kQBytes;             // kStages K tiles
 constexpr uint32_t kVOff = kKOff + kStages * kKVBytes;      // kStages V tiles
-constexpr uint32_t kOOff = kVOff + kStages * kKVBytes;      // O staging tile for the TMA store
-constexpr uint32_t kBarOff = kOOff + kQBytes;
+constexpr uint32_t kBarOff = kVOff + kStages * kKVBytes;
 constexpr uint32_t kItemOff = kBarOff + 256;
 constexpr uint32_t kSmemBytes = kItemOff + kMaxItems * 32 + 1024;   // + item table + alignment slack
 constexpr uint32_t kTmemCols = 256;                         // power of two, >= 32
@@ -113,8 +117,7 @@ struct Bars {
   uint64_t p_full[2];    // every softmax thread has written P of tile g (128 arrivals)
   uint64_t pv_done[2];   // PV of tile g done (tcgen05.commit)
   uint64_t mma_done;
-  uint64_t o_ready;      // every softmax thread has written its row of the O staging tile (128 arrivals)
-  uint64_t o_free;       // the last TMA store has finished reading the staging tile
+  uint64_t o_ready;      // every softmax thread has written its row of O into the item's Q buffer (128 arrivals)
   uint32_t tmem_base;
   int abort;
 };
@@ -252,7 +255,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     for (int i = 0; i < kStages; ++i) { mbar_init(&bars->kv_full[i], 1); mbar_init(&bars->kv_empty[i], 1); }
     mbar_init(&bars->mma_done, 1);
     mbar_init(&bars->o_ready, kBM);
-    mbar_init(&bars->o_free, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -272,16 +274,31 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_kc); tma_prefetch_desc(&tm_vc); tma_prefetch_desc(&tm_o);
       int g = 0, wi = 0;
+      int n_st = 0;              // O tiles stored so far (phases of o_ready)
+      int q_item0 = -1, q_item1 = -1;  // the item whose Q (then O) each buffer holds
+      // a whole 128-row O tile is staged by the softmax warps in its item's Q buffer; it leaves
+      // with one TMA store, and the buffer takes new Q only once the store has read it
+      auto store_o = [&](int u) -> bool {
+        const Item& it = items[u ? q_item1 : q_item0];
+        if (it.q_last != it.q0 + kBM - 1) return true;   // a partial tile was written row by row
+        if (!mbar_wait_bounded(&bars->o_ready, n_st & 1, abort_flag, kWaitNs)) return false;
+        tma_store_3d(&tm_o, smem + kQOff + u * kQBytes, 0, it.h, (int)((int64_t)it.b * n + it.q0));
+        tma_store_wait_read();
+        ++n_st;
+        return true;
+      };
       bool ok = true;
       for (int k = 0; ok && k < my_items; ++k) {
         const Item it = items[k];
         if (it.NT == 0) continue;
         const int64_t tok0 = (int64_t)it.b * n;
         const int qb = wi & 1;
-        if (wi >= 2 && !mbar_wait_bounded(&bars->q_empty[qb], ((wi - 2) >> 1) & 1, abort_flag, kWaitNs)) {
+        if (wi >= 2 && (!mbar_wait_bounded(&bars->q_empty[qb], ((wi - 2) >> 1) & 1, abort_flag, kWaitNs) ||
+                        !store_o(qb))) {
           ok = false;
           break;
         }
+        if (qb) q_item1 = k; else q_item0 = k;
         mbar_arrive_expect_tx(&bars->q_full[qb], kQBytes);
         tma_load_3d(smem + kQOff + qb * kQBytes, &tm_q, 0, it.h, (int)(tok0 + it.q0), &bars->q_full[qb]);
         ++wi;
@@ -299,11 +316,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           tma_load_3d(smem + kVOff + st * kKVBytes, bnd ? &tm_vc : &tm_v, 0, it.h, row, &bars->kv_full[st]);
         }
       }
+      // the last two items' O tiles
+      for (int u = max(0, wi - 2); ok && u < wi; ++u) ok = store_o(u & 1);
       if (!ok) *abort_flag = 1;
-      // drain: the last copies into each buffer must land before the CTA may exit
+      // drain: the last copies into each buffer must land, and the stores complete, before the CTA may exit
       for (int u = max(0, wi - 2); u < wi; ++u) mbar_wait_timeout(&bars->q_full[u & 1], (u >> 1) & 1, kWaitNs);
       for (int j = max(0, g - kStages); j < g; ++j)
         mbar_wait_timeout(&bars->kv_full[j % kStages], (j / kStages) & 1, kWaitNs);
+      tma_store_wait_all();
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
@@ -326,11 +346,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         return true;
       };
       int g = 0, wi = 0;
-      bool pend_first = false;
+      bool pend = false, pend_first = false;   // PV(g - 1) not issued yet; it is its item's first tile
       bool ok = true;
       for (int k = 0; ok && k < my_items; ++k) {
         const Item it = items[k];
         if (it.NT == 0) continue;
+        // the previous item's last PV goes first: its epilogue must not wait for this item's loads
+        if (pend) {
+          if (!issue_pv(g - 1, pend_first)) { ok = false; break; }
+          pend = false;
+        }
         const int qb = wi & 1;
         if (!mbar_wait_bounded(&bars->q_full[qb], (wi >> 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
         const uint32_t sq = smem_u32(smem + kQOff + qb * kQBytes);
@@ -350,12 +375,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                       umma_desc_sw128(sk + kk * 32, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
           umma_commit(&bars->s_full[g & 1]);
           if (j == it.NT - 1) umma_commit(&bars->q_empty[qb]);  // Q free once the item's last QK is done
-          if (g >= 1 && !issue_pv(g - 1, pend_first)) { ok = false; break; }
+          if (pend && !issue_pv(g - 1, pend_first)) { ok = false; break; }
+          pend = true;
           pend_first = (j == 0);
         }
         ++wi;
       }
-      if (ok && g >= 1) ok = issue_pv(g - 1, pend_first);
+      if (ok && pend) ok = issue_pv(g - 1, pend_first);
       if (!ok) *abort_flag = 1;
       umma_commit(&bars->mma_done);  // every MMA issued above has finished when this arrives
       mbar_wait_timeout(&bars->mma_done, 0, kWaitNs);
@@ -366,11 +392,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const float sl2 = a.scale * kLog2e;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     const uint32_t o_tmem = lane_base + kOCol;
-    uint8_t* orow = smem + kOOff + r * 128;   // this row of the O staging tile
     const int sw = r & 7;
-    int g = 0;
+    int g = 0, wi = 0;   // key tiles and non-empty items so far (item wi's Q is in buffer wi & 1)
     bool ok = true;
-    int n_stores = 0;   // TMA stores of the staging tile issued so far (phases of o_ready / o_free)
     // wait for the PV of tile gg (barrier gg & 1, its phase gg >> 1; verdict warp-uniform)
     auto wait_pv = [&](int gg) -> bool {
       return __all_sync(0xffffffffu,
@@ -499,19 +523,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       if (!wait_pv(g - 1)) { ok = false; break; }
       tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      const bool whole = it.q_last == it.q0 + kBM - 1;   // a full tile leaves through one TMA store
-      if (whole && n_stores > 0) {
-        // the staging tile is free once the previous store has read it
-        if (r == 0) {
-          tma_store_wait_read();
-          mbar_arrive(&bars->o_free);
-        }
-        if (!__all_sync(0xffffffffu,
-                        mbar_wait_bounded(&bars->o_free, (n_stores - 1) & 1, abort_flag, kWaitNs))) {
-          ok = false;
-          break;
-        }
-      }
+      // a full tile is staged in the item's Q buffer (its last QK finished before this PV did)
+      // and leaves through one TMA store issued by the producer
+      const bool whole = it.q_last == it.q0 + kBM - 1;
+      uint8_t* orow = smem + kQOff + (wi & 1) * kQBytes + r * 128;
+      ++wi;
       uint4* dst = reinterpret_cast<uint4*>(O + ((tok0 + i) * H + it.h) * kDH);
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
@@ -534,19 +550,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       if (whole) {
         fence_async_smem();
         mbar_arrive(&bars->o_ready);
-        if (warp == 0) {
-          // one thread issues the store once every row is in place; warp 0 leaves together on a timeout
-          bool okw = true;
-          if (lane == 0) {
-            okw = mbar_wait_bounded(&bars->o_ready, n_stores & 1, abort_flag, kWaitNs);
-            if (okw) tma_store_3d(&tm_o, smem + kOOff, 0, it.h, (int)(tok0 + it.q0));
-          }
-          if (!__shfl_sync(0xffffffffu, okw, 0)) {
-            ok = false;
-            break;
-          }
-        }
-        ++n_stores;
       }
       if (row_ok && a.lse)
         a.lse[((int64_t)it.b * H + it.h) * n + i] = l_run > 0.f ? (m_ref + __log2f(l_run)) * kLn2 : -INFINITY;
@@ -555,8 +558,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       *abort_flag = 1;
       raise_status(a.status, ATTAMBA_DEV_TIMEOUT);
     }
-    // the stores must be complete before the CTA's shared memory goes away
-    if (r == 0 && n_stores > 0) tma_store_wait_all();
   }
 
   tc_fence_before();

@@ -8,14 +8,23 @@
 // reached only through the leading tokens.
 //
 // Two stream-ordered launches, no inter-CTA waiting:
-//   decode_attn_kernel    per (split, head, sequence): the last split first runs the
-//                         SSM step of the head's channels (reset at a chunk start,
-//                         state [2,B,N,D] read and written coalesced, k_t / v_t into
-//                         ring slot t mod L and, at a chunk end, into the boundary
-//                         list); every split then streams its share of the
-//                         (boundaries below the window) + (window) keys with
-//                         16-byte loads, 8 lanes per key row, fp32 online softmax,
-//                         and writes (max, sum, unnormalised output) to the workspace
+//   decode_attn_kernel    per (split, head, sequence), warps 0-3 compute and warp 4
+//                         copies.  The last split first runs the SSM step of the
+//                         head's channels (reset at a chunk start, state [2,B,N,D]
+//                         read and written coalesced, k_t / v_t into ring slot
+//                         t mod L and, at a chunk end, into the boundary list) while
+//                         warp 4 finds, with a 32-way search of the sorted boundary
+//                         positions, how many boundaries lie below the window.  The
+//                         split's keys -- (boundaries below the window) then
+//                         (window) -- are contiguous row runs of the cache (at most
+//                         three per 64-key stage: boundary rows, then the ring
+//                         before and after its wrap), so one thread streams them
+//                         into a ring of shared-memory stages with bulk async
+//                         copies (cp.async.bulk, completion on an mbarrier) and
+//                         keeps several stages in flight per CTA; the compute warps
+//                         read each key row as 8 lanes x 16 bytes, keep an fp32
+//                         online softmax, and write (max, sum, unnormalised output)
+//                         to the workspace
 //   decode_combine_kernel per (sequence, head): merges the splits, writes o_t,
 //                         and advances pos / nb
 // The step is bound by streaming the cached K/V from HBM.
@@ -38,9 +47,52 @@ static __device__ __align__(256) float g_decode_scratch[kNoAllocScratchFloats];
 
 namespace {
 constexpr int kDH = 64;
-constexpr int kAttnThreads = 128;
-constexpr int kUnroll = 4;
+constexpr int kComputeThreads = 128;                      // warps 0-3
+constexpr int kAttnThreads = kComputeThreads + 32;        // + warp 4, the copy warp
+constexpr int kUnroll = 4;                                // keys per lane group and stage
+constexpr int kStageKeys = 16 * kUnroll;                  // 4 warps x 4 lane groups x kUnroll
+#ifndef ATTAMBA_DECODE_STAGES
+#define ATTAMBA_DECODE_STAGES 4
+#endif
+constexpr int kStages = ATTAMBA_DECODE_STAGES;
+constexpr uint32_t kRowBytes = kDH * 2;                   // one bf16 key or value row
+constexpr uint32_t kStageBytes = kStageKeys * kRowBytes;  // per tensor
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+struct DecodeBars {
+  uint64_t full[kStages];    // the stage's K and V rows have landed (transaction count)
+  uint64_t empty[kStages];   // the four compute warps have read the stage
+  int nbb;                   // boundaries below the window
+  int abort;
+};
+constexpr uint32_t kSmemBytes = 2 * kStages * kStageBytes + sizeof(DecodeBars);
+// CTAs per SM that the stages allow (about 227 KB of shared memory per SM), for the register budget
+constexpr int kMinBlocks = (int)((220u * 1024u) / (kSmemBytes + 2048u)) < 8 ? (int)((220u * 1024u) / (kSmemBytes + 2048u)) : 8;
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// Number of entries of the ascending row p[0, n) that are below v, by all 32 lanes:
+// each round probes 32 evenly spaced entries and keeps the gap where the answer lies.
+__device__ __forceinline__ int count_below_warp(const int32_t* p, int n, int v, int lane) {
+  int l = 0, h = n;   // the answer lies in [l, h]
+  while (l < h) {
+    const int step = (h - l + 31) >> 5;
+    const int idx = l + lane * step;
+    const bool below = idx < h && p[idx] < v;
+    const int c = __popc(__ballot_sync(0xffffffffu, below));
+    if (c == 0) break;                       // p[l] >= v: the answer is l
+    const int nl = l + (c - 1) * step + 1;   // p[l + (c - 1) step] < v
+    h = min(h, l + c * step);                // p[l + c step] >= v, or the end
+    l = nl;
+  }
+  return l;
+}
 
 __device__ __forceinline__ bool chunk_starts_at(int t, int P, int o) {
   return t == 0 || (t >= o && (t - o) % P == 0);
@@ -108,43 +160,96 @@ __device__ __forceinline__ void bf16x8_to_f(const uint4& u, float (&f)[8]) {
 }
 
 template <int kNS>
-__global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kAttnThreads, kMinBlocks) decode_attn_kernel(DecodeArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(smem);
+  __nv_bfloat16* Vs = reinterpret_cast<__nv_bfloat16*>(smem + kStages * kStageBytes);
+  DecodeBars* bars = reinterpret_cast<DecodeBars*>(smem + 2 * kStages * kStageBytes);
   const attamba_cache_t& c = a.c;
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // The last split of (b, h) holds the newest key (position t): it first runs the SSM step of
-  // the head's 64 channels for both SSMs (one per thread), which writes k_t, v_t into the ring.
-  // No other block reads that slot (it held position t - L, now outside the window), and the
-  // boundary appended at a chunk end lies inside the window, so no other split reads it either.
-  if (split == a.splits - 1) {
-    ssm_step<kNS>(a, threadIdx.x >> 6, b, h * kDH + (threadIdx.x & 63));
-    __syncthreads();
-  }
-  const int g = lane >> 3;          // key group within the warp
-  const int e8 = (lane & 7) * 8;    // head-dim slice of this lane
   const int L = c.L, cap = c.cap;
   const int t = c.pos[b];
   const int lo = max(0, t - L + 1);
-  const int nw = t + 1 - lo;
-  // boundaries strictly below the window
-  const int32_t* bp = c.bpos + (size_t)b * cap;
-  int l0 = 0, h0 = min(max(c.nb[b], 0), cap);
-  while (l0 < h0) {
-    const int mid = (l0 + h0) >> 1;
-    if (bp[mid] < lo) l0 = mid + 1; else h0 = mid;
+  if (warp == 4) {
+    if (lane == 0) {
+      for (int i = 0; i < kStages; ++i) {
+        mbar_init(&bars->full[i], 1);
+        mbar_init(&bars->empty[i], 4);
+      }
+      bars->abort = 0;
+      fence_mbar_init();
+    }
+    // boundaries strictly below the window (the entry the SSM step may append lies past nb)
+    const int nbb = count_below_warp(c.bpos + (size_t)b * cap, min(max(c.nb[b], 0), cap), lo, lane);
+    if (lane == 0) bars->nbb = nbb;
+  } else if (split == a.splits - 1) {
+    // The last split of (b, h) holds the newest key (position t): it first runs the SSM step of
+    // the head's 64 channels for both SSMs (one per thread), which writes k_t, v_t into the ring.
+    // No other block reads that slot (it held position t - L, now outside the window), and the
+    // boundary appended at a chunk end lies inside the window, so no other split reads it either.
+    ssm_step<kNS>(a, threadIdx.x >> 6, b, h * kDH + (threadIdx.x & 63));
+    // the copy warp reads the ring through the async proxy
+    asm volatile("fence.proxy.async.global;" ::: "memory");
   }
-  const int nbb = l0;
-  const int nkeys = nbb + nw;
+  __syncthreads();
+  const int nbb = bars->nbb;
+  const int nkeys = nbb + (t + 1 - lo);
   const int per = (nkeys + a.splits - 1) / a.splits;
   const int kb = split * per;
   const int ke = min(nkeys, kb + per);
-
+  const int nst = ke > kb ? (ke - kb + kStageKeys - 1) / kStageKeys : 0;
   const size_t bh = (size_t)b * c.H + h;
-  const __nv_bfloat16* Kb = static_cast<const __nv_bfloat16*>(c.Kb) + bh * cap * kDH + e8;
-  const __nv_bfloat16* Vb = static_cast<const __nv_bfloat16*>(c.Vb) + bh * cap * kDH + e8;
-  const __nv_bfloat16* Kr = static_cast<const __nv_bfloat16*>(c.Kr) + bh * L * kDH + e8;
-  const __nv_bfloat16* Vr = static_cast<const __nv_bfloat16*>(c.Vr) + bh * L * kDH + e8;
+  volatile int* abort_flag = &bars->abort;
 
+  if (warp == 4) {
+    // ------------------------------------------------------------ copy warp
+    if (lane == 0) {
+      const uint8_t* Kb = static_cast<const uint8_t*>(c.Kb) + bh * cap * kRowBytes;
+      const uint8_t* Vb = static_cast<const uint8_t*>(c.Vb) + bh * cap * kRowBytes;
+      const uint8_t* Kr = static_cast<const uint8_t*>(c.Kr) + bh * L * kRowBytes;
+      const uint8_t* Vr = static_cast<const uint8_t*>(c.Vr) + bh * L * kRowBytes;
+      bool ok = true;
+      int s = 0;
+      for (; s < nst; ++s) {
+        const int st = s % kStages;
+        if (s >= kStages && !mbar_wait_bounded(&bars->empty[st], ((s / kStages) - 1) & 1, abort_flag, kWaitNs)) {
+          ok = false;
+          break;
+        }
+        const int k0 = kb + s * kStageKeys, k1 = min(ke, k0 + kStageKeys);
+        uint64_t* bar = &bars->full[st];
+        mbar_arrive_expect_tx(bar, (uint32_t)(k1 - k0) * 2 * kRowBytes);
+        uint8_t* dK = reinterpret_cast<uint8_t*>(Ks) + st * kStageBytes;
+        uint8_t* dV = reinterpret_cast<uint8_t*>(Vs) + st * kStageBytes;
+        // boundary rows k0 .. min(k1, nbb) - 1
+        const int b1 = min(k1, nbb);
+        if (b1 > k0) {
+          bulk_g2s(dK, Kb + (size_t)k0 * kRowBytes, (uint32_t)(b1 - k0) * kRowBytes, bar);
+          bulk_g2s(dV, Vb + (size_t)k0 * kRowBytes, (uint32_t)(b1 - k0) * kRowBytes, bar);
+        }
+        // window keys: key k >= nbb is position lo + (k - nbb), in ring slot (lo + k - nbb) mod L
+        for (int k = max(k0, nbb); k < k1;) {
+          const int slot = (lo + (k - nbb)) % L;
+          const int cnt = min(k1 - k, L - slot);
+          bulk_g2s(dK + (k - k0) * kRowBytes, Kr + (size_t)slot * kRowBytes, (uint32_t)cnt * kRowBytes, bar);
+          bulk_g2s(dV + (k - k0) * kRowBytes, Vr + (size_t)slot * kRowBytes, (uint32_t)cnt * kRowBytes, bar);
+          k += cnt;
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        // copies may still be in flight into the stages: they must land before the CTA exits
+        for (int j = max(0, s - kStages); j < s; ++j)
+          mbar_wait_timeout(&bars->full[j % kStages], (j / kStages) & 1, kWaitNs);
+      }
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- compute warps 0-3
+  const int g = lane >> 3;          // key group within the warp
+  const int e8 = (lane & 7) * 8;    // head-dim slice of this lane
   float qf[8];
   {
     const uint4 qu = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + bh * kDH + e8);
@@ -157,30 +262,30 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(DecodeArgs a)
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 
-  // Keys are processed in sweeps of 16 (4 warps x 4 key groups) x kUnroll; two register
-  // buffers alternate so one sweep's loads are in flight while the other is computed.
-  auto load_sweep = [&](int kk, uint4 (&kr)[kUnroll], uint4 (&vr)[kUnroll]) {
+  bool ok = true;
+  for (int s = 0; s < nst; ++s) {
+    const int st = s % kStages;
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars->full[st], (s / kStages) & 1, abort_flag, kWaitNs))) {
+      ok = false;
+      break;
+    }
+    const int cnt = min(ke - kb - s * kStageKeys, kStageKeys);
+    const __nv_bfloat16* ks = Ks + st * (kStageKeys * kDH) + e8;
+    const __nv_bfloat16* vs = Vs + st * (kStageKeys * kDH) + e8;
+    uint4 kr[kUnroll], vr[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const int k = kk + u * 16 + g;
-      if (k < ke) {
-        if (k < nbb) {
-          kr[u] = __ldg(reinterpret_cast<const uint4*>(Kb + (size_t)k * kDH));
-          vr[u] = __ldg(reinterpret_cast<const uint4*>(Vb + (size_t)k * kDH));
-        } else {
-          // the ring is written during the step (slot of t): read it through L2, not the
-          // read-only path
-          const int slot = (lo + (k - nbb)) % L;
-          kr[u] = __ldcg(reinterpret_cast<const uint4*>(Kr + (size_t)slot * kDH));
-          vr[u] = __ldcg(reinterpret_cast<const uint4*>(Vr + (size_t)slot * kDH));
-        }
+      const int row = u * 16 + warp * 4 + g;
+      if (row < cnt) {
+        kr[u] = *reinterpret_cast<const uint4*>(ks + row * kDH);
+        vr[u] = *reinterpret_cast<const uint4*>(vs + row * kDH);
       } else {
         kr[u] = make_uint4(0, 0, 0, 0);
         vr[u] = make_uint4(0, 0, 0, 0);
       }
     }
-  };
-  auto compute_sweep = [&](int kk, const uint4 (&kr)[kUnroll], const uint4 (&vr)[kUnroll]) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars->empty[st]);   // this warp's rows of the stage are in registers
     float sc[kUnroll];
     float mt = -INFINITY;
 #pragma unroll
@@ -193,7 +298,7 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(DecodeArgs a)
       dot += __shfl_xor_sync(0xffffffffu, dot, 1);
       dot += __shfl_xor_sync(0xffffffffu, dot, 2);
       dot += __shfl_xor_sync(0xffffffffu, dot, 4);
-      sc[u] = (kk + u * 16 + g < ke) ? dot : -INFINITY;
+      sc[u] = (u * 16 + warp * 4 + g < cnt) ? dot : -INFINITY;
       mt = fmaxf(mt, sc[u]);
     }
     const float m_new = fmaxf(m, mt);
@@ -213,22 +318,10 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(DecodeArgs a)
       }
       m = m_new;
     }
-  };
-  constexpr int kSweep = 16 * kUnroll;
-  uint4 kA[kUnroll], vA[kUnroll], kB[kUnroll], vB[kUnroll];
-  int kk = kb + warp * 4;
-  if (kk < ke) load_sweep(kk, kA, vA);
-  while (kk < ke) {
-    const bool more = kk + kSweep < ke;
-    if (more) load_sweep(kk + kSweep, kB, vB);
-    compute_sweep(kk, kA, vA);
-    if (!more) break;
-    kk += kSweep;
-    const bool more2 = kk + kSweep < ke;
-    if (more2) load_sweep(kk + kSweep, kA, vA);
-    compute_sweep(kk, kB, vB);
-    if (!more2) break;
-    kk += kSweep;
+  }
+  if (!ok) {
+    *abort_flag = 1;
+    if (lane == 0) raise_status(a.status, ATTAMBA_DEV_TIMEOUT);
   }
 
   // merge the four key groups of the warp (lanes with the same slice: xor 8, 16)
@@ -247,14 +340,15 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(DecodeArgs a)
     }
     m = mn;
   }
-  // merge the four warps through shared memory
+  // merge the four warps through shared memory (a barrier of the compute warps only: every one
+  // of them gets here, a timed-out wait included)
   __shared__ float s_m[4], s_l[4], s_acc[4][kDH];
   if (lane < 8) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) s_acc[warp][e8 + i] = acc[i];
     if (lane == 0) { s_m[warp] = m; s_l[warp] = l; }
   }
-  __syncthreads();
+  asm volatile("bar.sync 1, %0;" ::"n"(kComputeThreads) : "memory");
   if (threadIdx.x < kDH) {
     const int e = threadIdx.x;
     float M = -INFINITY;
@@ -300,7 +394,10 @@ __global__ void __launch_bounds__(kDH) decode_combine_kernel(DecodeArgs a) {
 
 int32_t decode_splits(const attamba_cache_t& c) {
   const int64_t bh = (int64_t)c.B * c.H;
-  const int64_t target = 8 * 148;
+#ifndef ATTAMBA_DECODE_TARGET
+#define ATTAMBA_DECODE_TARGET (8 * 148)
+#endif
+  const int64_t target = ATTAMBA_DECODE_TARGET;
   int64_t sp = (target + bh - 1) / bh;
   const int64_t max_sp = ((int64_t)c.cap + c.L) / 128;
   if (sp > max_sp) sp = max_sp;
@@ -336,10 +433,14 @@ size_t decode_workspace_bytes(const attamba_cache_t& c) {
 }
 
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s) {
+  const void* k = a.c.N == 32 ? reinterpret_cast<const void*>(decode_attn_kernel<32>)
+                              : reinterpret_cast<const void*>(decode_attn_kernel<16>);
+  cudaError_t e = raise_smem_limit(k, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
   if (a.c.N == 32)
-    decode_attn_kernel<32><<<dim3(a.splits, a.c.H, a.c.B), kAttnThreads, 0, s>>>(a);
+    decode_attn_kernel<32><<<dim3(a.splits, a.c.H, a.c.B), kAttnThreads, kSmemBytes, s>>>(a);
   else
-    decode_attn_kernel<16><<<dim3(a.splits, a.c.H, a.c.B), kAttnThreads, 0, s>>>(a);
+    decode_attn_kernel<16><<<dim3(a.splits, a.c.H, a.c.B), kAttnThreads, kSmemBytes, s>>>(a);
   decode_combine_kernel<<<a.c.B * a.c.H, kDH, 0, s>>>(a);
   return cudaGetLastError();
 }
