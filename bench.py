@@ -8,6 +8,10 @@ bf16): chunk index -> KV-SSM scan (K and V) -> chunk-masked attention, three
 C-ABI calls on inputs already resident in HBM.  L2 is flushed between steps
 (a 256 MiB write, outside the per-step events).  Each rank runs its own batch
 (weak scaling, no collective on the data path); the time is the max over ranks.
+Each timed step is bracketed by two CUDA events on the launching stream (the
+scan and the attention are programmatic dependent launches, so nothing is
+recorded between the calls); a second pass of the same steps with events
+between the calls gives each kernel's time for the roofline.
 
 --impl reference times the CPU oracle (float64 numpy, test infrastructure) on
 this host's cores on a bounded sample of the same workload.
@@ -384,18 +388,21 @@ def run_ours(args, ws, rank, local):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def step(events=None):
+        """One step: chunk_index, kv_ssm_scan, chunk_attn_fwd.  Two events bracket the step; four
+        also split it per call (an event between two calls keeps the second call's launch from
+        overlapping the first call's tail, so the split sums to a little more than the step)."""
         if events:
             events[0].record(stream)
         pf.index_step(None, cfg.P, cfg.offset, cfg.L, mode)
-        if events:
+        if events and len(events) == 4:
             events[1].record(stream)
         pf.scan_step(g["x"], g["dt_k"], g["dt_v"], g["bias_k"], g["bias_v"], g["A_k"], g["A_v"], g["B_k"],
                      g["C_k"], g["B_v"], g["C_v"])
-        if events:
+        if events and len(events) == 4:
             events[2].record(stream)
         pf.attn_step(g["q"], inp["scale"])
         if events:
-            events[3].record(stream)
+            events[-1].record(stream)
 
     sampler = ClockSampler(local) if rank == 0 else None
     t_w = time.perf_counter()
@@ -419,7 +426,9 @@ def run_ours(args, ws, rank, local):
     scan_exps = 2.0 * T * D * N
     index_bytes = T * 8 + nch * 8
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    # timed region: K steps, each bracketed by two events on the launching stream (the L2 flush
+    # between steps lies outside them)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     barrier(ws)
     torch.cuda.synchronize()
     if sampler:
@@ -430,11 +439,17 @@ def run_ours(args, ws, rank, local):
     torch.cuda.synchronize()
     barrier(ws)
     clocks = sampler.stop() if sampler else None
-
-    per = np.array([[evs[k][j].elapsed_time(evs[k][j + 1]) for j in range(3)] for k in range(args.steps)])  # ms
-    step_ms = per.sum(axis=1)
+    step_ms = np.array([evs[k][0].elapsed_time(evs[k][1]) for k in range(args.steps)])
     ms = max_over_ranks(float(step_ms.mean()), ws)
     value = job_throughput(ws, T, ms)
+
+    # per-call split (roofline of each kernel): the same K steps again with events between the calls
+    evk = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)
+        step(evk[k])
+    torch.cuda.synchronize()
+    per = np.array([[evk[k][j].elapsed_time(evk[k][j + 1]) for j in range(3)] for k in range(args.steps)])  # ms
 
     # end to end through the public API with host buffers: pinned H2D of the step's activations,
     # the three calls, D2H of the output

@@ -242,7 +242,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (tid == 0) raise_status(a.status, ATTAMBA_DEV_TIMEOUT);
     return;
   }
-  for (int k = tid; k < my_items; k += kThreads) items[k] = decode_item(a, blockIdx.x + k * gridDim.x, n_qt);
   if (warp == 4 && lane == 0) {
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->q_full[b], 1);
@@ -262,6 +261,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  // launched as a programmatic dependent of the previous kernel in the stream, whose outputs may be
+  // this kernel's inputs: the set-up above reads none, everything below waits for that grid
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  for (int k = tid; k < my_items; k += kThreads) items[k] = decode_item(a, blockIdx.x + k * gridDim.x, n_qt);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -648,8 +651,17 @@ cudaError_t launch_chunk_attn_bf16(const AttnArgs& a, cudaStream_t s) {
   int64_t grid = items < (int64_t)kCtasPerSm * sms ? items : (int64_t)kCtasPerSm * sms;
   if ((items + grid - 1) / grid > kMaxItems) grid = (items + kMaxItems - 1) / kMaxItems;
   if (grid > 2147483647) return cudaErrorInvalidValue;
-  chunk_attn_bf16_kernel<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tkc, tvc, to, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, chunk_attn_bf16_kernel, tq, tk, tv, tkc, tvc, to, a);
 }
 
 cudaError_t launch_chunk_attn_f32(const AttnArgs& a, cudaStream_t s) {

@@ -26,7 +26,10 @@
 //                         online softmax, and write (max, sum, unnormalised output)
 //                         to the workspace
 //   decode_combine_kernel per (sequence, head): merges the splits, writes o_t,
-//                         and advances pos / nb
+//                         and advances pos / nb; launched as a programmatic
+//                         dependent of the attention kernel (its launch overlaps
+//                         that kernel's tail; it waits for the grid's completion
+//                         before reading the workspace)
 // The step is bound by streaming the cached K/V from HBM.
 #include <mutex>
 
@@ -323,6 +326,9 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) decode_attn_kernel(D
     *abort_flag = 1;
     if (lane == 0) raise_status(a.status, ATTAMBA_DEV_TIMEOUT);
   }
+  // the combine may be scheduled once every CTA is past its key loop (it still waits for this
+  // grid to complete before it reads the workspace)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // merge the four key groups of the warp (lanes with the same slice: xor 8, 16)
 #pragma unroll
@@ -367,6 +373,9 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) decode_attn_kernel(D
 }
 
 __global__ void __launch_bounds__(kDH) decode_combine_kernel(DecodeArgs a) {
+  // launched as a programmatic dependent of decode_attn_kernel: wait for that grid's completion
+  // and memory before reading what it wrote
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const attamba_cache_t& c = a.c;
   const int bh = blockIdx.x;
   const int e = threadIdx.x;
@@ -441,8 +450,20 @@ cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s) {
     decode_attn_kernel<32><<<dim3(a.splits, a.c.H, a.c.B), kAttnThreads, kSmemBytes, s>>>(a);
   else
     decode_attn_kernel<16><<<dim3(a.splits, a.c.H, a.c.B), kAttnThreads, kSmemBytes, s>>>(a);
-  decode_combine_kernel<<<a.c.B * a.c.H, kDH, 0, s>>>(a);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // the combine's launch overlaps the attention kernel's tail (programmatic dependent launch)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(a.c.B * a.c.H));
+  cfg.blockDim = dim3(kDH);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_combine_kernel, a);
 }
 
 }  // namespace attamba

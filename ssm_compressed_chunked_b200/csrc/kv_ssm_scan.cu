@@ -205,6 +205,9 @@ __global__ void __launch_bounds__(kScanThreads, MINB) kv_ssm_scan_kernel(ScanArg
   constexpr int kNP = NS / 2;
   __shared__ __align__(16) float sBC[kStageTokens][2 * kNS];  // B then C of each staged token
   __shared__ int sCu[kMaxChunksPerBlock + 1];                 // chunk starts of this block
+  // launched as a programmatic dependent of the previous kernel in the stream: its outputs may be
+  // this kernel's inputs, so nothing is read before that grid has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   const int s = blockIdx.z;
   const int D = p.D;  // T * D < 2^31 (checked by the host): 32-bit element offsets
@@ -316,12 +319,20 @@ cudaError_t launch_scan(attamba_dtype_t dtype, const ScanArgs& a, cudaStream_t s
   if (cpb > kMaxChunksPerBlock) cpb = kMaxChunksPerBlock;
   if ((a.n_chunks + cpb - 1) / cpb > 65535) return cudaErrorInvalidValue;
   dim3 grid((a.D / CPT + kScanThreads - 1) / kScanThreads, (unsigned)((a.n_chunks + cpb - 1) / cpb), 2);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kScanThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (dtype == ATTAMBA_BF16)
-    kv_ssm_scan_kernel<__nv_bfloat16, CPT, NS, NS == 16 ? ATTAMBA_SCAN_POLY_PAIRS : 0, MINB, SPLIT_X>
-        <<<grid, kScanThreads, 0, s>>>(a, (int32_t)cpb);
-  else
-    kv_ssm_scan_kernel<float, CPT, NS, 0, MINB, SPLIT_X><<<grid, kScanThreads, 0, s>>>(a, (int32_t)cpb);
-  return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, kv_ssm_scan_kernel<__nv_bfloat16, CPT, NS, NS == 16 ? ATTAMBA_SCAN_POLY_PAIRS : 0, MINB, SPLIT_X>,
+                              a, (int32_t)cpb);
+  return cudaLaunchKernelEx(&cfg, kv_ssm_scan_kernel<float, CPT, NS, 0, MINB, SPLIT_X>, a, (int32_t)cpb);
 }
 }  // namespace
 
