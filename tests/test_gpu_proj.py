@@ -54,3 +54,47 @@ def test_proj_gemm_skips_columns_no_segment_names():
     ref = OP.project(f64(X.cpu()), f64(W.cpu()))
     _check(a.cpu(), ref[:, 8:24], X.cpu(), W.cpu()[8:24], "a")
     _check(b.cpu(), ref[:, 64:72], X.cpu(), W.cpu()[64:72], "b")
+
+
+def test_proj_gemm_more_tiles_than_resident_pairs():
+    """320 output tiles of 256 x 256 against 74 resident CTA pairs: every pair runs several tiles, so
+    both TMEM accumulators are reused and the stage ring wraps many times."""
+    M, K, widths = 8192, 128, [1024, 1024, 512]
+    gen = torch.Generator().manual_seed(11)
+    Nout = sum(widths)
+    X = torch.randn(M, K, generator=gen).to(torch.bfloat16)
+    W = (torch.randn(Nout, K, generator=gen) / K ** 0.5).to(torch.bfloat16)
+    outs, c = [], 0
+    for w in widths:
+        outs.append((torch.full((M, w), float("nan"), dtype=torch.bfloat16, device="cuda"), c))
+        c += w
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    A.proj_gemm(X.cuda(), W.cuda(), outs, status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ref = OP.split(OP.project(f64(X), f64(W)), widths)
+    for k, ((t, _), r) in enumerate(zip(outs, ref)):
+        _check(t.cpu(), r, X, W[sum(widths[:k]):sum(widths[:k + 1])], f"segment {k}")
+
+
+def test_proj_gemm_layer_size_sampled_rows():
+    """The layer's input projections at the bench size (M = 4 x 4096 tokens, K = 1024, seven
+    segments): 96 sampled rows against the oracle's float64 product of those rows."""
+    M, K, widths = 16384, 1024, [1024, 1024, 1024, 16, 16, 16, 16]
+    gen = torch.Generator().manual_seed(12)
+    Nout = sum(widths)
+    X = torch.randn(M, K, generator=gen).to(torch.bfloat16)
+    W = (torch.randn(Nout, K, generator=gen) / K ** 0.5).to(torch.bfloat16)
+    outs, c = [], 0
+    for w in widths:
+        outs.append((torch.full((M, w), float("nan"), dtype=torch.bfloat16, device="cuda"), c))
+        c += w
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    A.proj_gemm(X.cuda(), W.cuda(), outs, status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    rows = torch.randperm(M, generator=gen)[:96].sort().values
+    Xs = X[rows]
+    ref = OP.split(OP.project(f64(Xs), f64(W)), widths)
+    for k, ((t, _), r) in enumerate(zip(outs, ref)):
+        _check(t.cpu()[rows], r, Xs, W[sum(widths[:k]):sum(widths[:k + 1])], f"segment {k}")
