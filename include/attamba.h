@@ -23,7 +23,10 @@
  *     16-byte aligned.  The library allocates nothing and keeps no state
  *     between calls; it is thread-safe.
  *   - Every call is asynchronous on the given stream (a cudaStream_t; NULL is
- *     the legacy default stream) and never synchronizes.
+ *     the legacy default stream) and never synchronizes.  The scans and the
+ *     bf16 attention are programmatic dependent launches: they may start while
+ *     the previous kernel in the stream is finishing, but read no input before
+ *     that kernel has completed, so stream order holds as for any launch.
  *   - Arguments the host can check are checked before any launch; a bad one
  *     returns ATTAMBA_ERR_INVALID_ARG (or ATTAMBA_ERR_UNSUPPORTED for a shape
  *     or dtype outside the supported set) and launches nothing.
