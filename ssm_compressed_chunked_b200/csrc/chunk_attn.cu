@@ -18,18 +18,21 @@
 //              operands in shared memory) into TMEM, then O += P V (M128 N64
 //              K64, P read from TMEM, V from shared memory)
 //   warps 0-3  softmax, one query row per thread: one tcgen05.ld for its S row,
-//              masking only where the row's key range cuts the tile, 32-column
-//              chunks outside every row's range skipped, online max/sum in
-//              fp32, P as bf16 pairs back into TMEM with one tcgen05.st
+//              masking (a 64-bit column mask, one bit test and one select per
+//              column) only where the row's key range cuts the tile, 32-column
+//              chunks outside every row's range skipped, fp32 sums, P as bf16
+//              pairs back into TMEM with one tcgen05.st
 // TMEM per CTA (256 columns): S in two buffers of 64, P in two of 32, O 64.
 // With S and P double-buffered the QK of tile g + 1 and the PV of tile g - 1
 // run while the softmax works on tile g; the softmax waits only for the PV
 // that last read the P buffer it is about to fill (tile g - 2).  Because the
 // four softmax warps can then drift up to two tiles apart, every barrier they
 // arrive on exists per buffer.  O accumulates in TMEM across an item's tiles;
-// P uses a reference max that is raised (and O, l rescaled in TMEM) only when
-// a row's max grows by more than 2^8, so P <= 2^8 and the rescale is rare; the
-// final O / l is exact whatever reference was used.  A full 128-row tile of O
+// P = exp2(s - m_ref) against a per-row reference that only has to keep P
+// finite: it is the row max of the first tile where the row has keys, and it
+// moves to the current row max (P recomputed, O and l rescaled in TMEM) only
+// when a tile's row sum exceeds 2^16 or overflows, so the row max is computed
+// on few tiles; the final O / l is exact whatever reference was used.  A full 128-row tile of O
 // is staged (128-byte swizzle) in its item's own Q buffer, whose last reader,
 // the item's last QK, has finished by then, and leaves with one TMA store; the
 // producer issues the store and refills the buffer with the Q of the item two
@@ -39,9 +42,11 @@
 // wait for the next item's loads.
 //
 // Measured limits (B200, bench workload): the exponentials of a 64-column
-// tile cost 512 cycles of the multi-function unit per warp, so two CTAs per SM
-// keep it about 60% busy; the rest of a tile's time is barrier and TMEM
-// latency.  A third CTA does not fit (TMEM, shared memory); eight softmax
+// tile cost 512 cycles of the multi-function unit per warp; with two softmax
+// warps per SM sub-partition the tile's other instructions (about half of them
+// on the integer/logic pipe) and the barrier and TMEM latencies set the pace,
+// so each instruction taken out of the tile loop shows: the column mask and
+// the on-demand row max took 78.5 us to 70.6 us.  A third CTA does not fit (TMEM, shared memory); eight softmax
 // warps with the 16-lane TMEM shapes, 128-key tiles, and moving a share of the
 // exponentials to an FMA-pipe polynomial all measured slower.
 //
@@ -99,7 +104,6 @@ constexpr uint32_t kOCol = 3 * kBN;                         // O: columns 192..2
 constexpr uint64_t kWaitNs = 4000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescale = 8.f;   // O is rescaled only when a row's max grows by more than 2^8
 static_assert(kOCol + kDH <= kTmemCols, "TMEM columns");
 
 // Double-buffered resources (Q, S, P) use barrier pairs: use u of the resource is
@@ -445,59 +449,88 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         mbar_arrive(&bars->s_empty[g & 1]);
         // row max of the raw scores over the valid columns [lo, hi); masked columns become -inf in place
         if (lo != 0 || hi != kBN) {
-          const unsigned span = (unsigned)(hi - lo);
+          // the valid columns as two 32-bit masks; each column is then one bit test and one select
+          const uint64_t below_hi = hi >= 64 ? ~0ull : ((1ull << hi) - 1);
+          const uint64_t below_lo = lo >= 64 ? ~0ull : ((1ull << lo) - 1);
+          const uint64_t valid = (hi > lo) ? (below_hi & ~below_lo) : 0ull;
+          const uint32_t v0 = (uint32_t)valid, v1 = (uint32_t)(valid >> 32);
 #pragma unroll
-          for (int c = 0; c < kBN; ++c)
-            if ((unsigned)(c - lo) >= span) sr[c] = 0xff800000u;
+          for (int c = 0; c < 32; ++c)
+            if (!(v0 & (1u << c))) sr[c] = 0xff800000u;
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (!(v1 & (1u << c))) sr[32 + c] = 0xff800000u;
         }
 #define S_(c) __uint_as_float(sr[c])
-        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+        // The reference m_ref only has to keep every P finite and of useful size; the final O / l
+        // is exact whatever it is.  So a tile is first exponentiated against the reference it
+        // finds, and the row max is taken only for a row with no reference yet, or when the row
+        // sum says some score rose more than 2^16 above it (or overflowed); then the row moves
+        // its reference to the max, P is recomputed and O and l are rescaled.
+        auto row_max = [&]() -> float {
+          float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < kBN; c += 8) {
-          mx0 = max3(mx0, S_(c), S_(c + 1));
-          mx1 = max3(mx1, S_(c + 2), S_(c + 3));
-          mx2 = max3(mx2, S_(c + 4), S_(c + 5));
-          mx3 = max3(mx3, S_(c + 6), S_(c + 7));
-        }
-        const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-        // lazy rescale: keep the reference max unless the row max rose by more than 2^8
-        const bool grow = (m_ref == -INFINITY) ? (mt > -INFINITY) : (mt > m_ref + kRescale);
-        const bool rescale = j > 0 && __any_sync(0xffffffffu, grow);
-        // factor that brings this row's O and l from the old reference to the new one
-        // (m_ref = -inf: O and l are still 0, the factor is 0)
-        const float fscale = (grow && j > 0) ? ex2(m_ref - mt) : 1.f;
-        if (grow) {
-          l_run *= fscale;
-          m_ref = mt;
-        }
-        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        const float2 sl2x2 = make_float2(sl2, sl2), negm = make_float2(-m_use, -m_use);
-        float2 sum0 = make_float2(0.f, 0.f), sum1 = make_float2(0.f, 0.f);
-        uint32_t pk[kBN / 2];
-#pragma unroll
-        for (int q = 0; q < kBN / 32; ++q) {
-          // a 32-column chunk outside every lane's [lo, hi) needs no exponentials
-          const bool need = __any_sync(0xffffffffu, lo < q * 32 + 32 && hi > q * 32);
-          if (need) {
-#pragma unroll
-            for (int c = 0; c < 32; c += 4) {
-              float2 e0 = ffma2(make_float2(S_(q * 32 + c), S_(q * 32 + c + 1)), sl2x2, negm);
-              float2 e1 = ffma2(make_float2(S_(q * 32 + c + 2), S_(q * 32 + c + 3)), sl2x2, negm);
-              e0 = make_float2(ex2(e0.x), ex2(e0.y));
-              e1 = make_float2(ex2(e1.x), ex2(e1.y));
-              sum0 = fadd2(sum0, e0);
-              sum1 = fadd2(sum1, e1);
-              pk[q * 16 + c / 2] = pack_bf16x2(e0.x, e0.y);
-              pk[q * 16 + c / 2 + 1] = pack_bf16x2(e1.x, e1.y);
-            }
-          } else {
-#pragma unroll
-            for (int c = 0; c < 16; ++c) pk[q * 16 + c] = 0u;
+          for (int c = 0; c < kBN; c += 8) {
+            mx0 = max3(mx0, S_(c), S_(c + 1));
+            mx1 = max3(mx1, S_(c + 2), S_(c + 3));
+            mx2 = max3(mx2, S_(c + 4), S_(c + 5));
+            mx3 = max3(mx3, S_(c + 6), S_(c + 7));
           }
+          return fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+        };
+        uint32_t pk[kBN / 2];
+        float tsum = 0.f;
+        auto exps = [&]() {
+          const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+          const float2 sl2x2 = make_float2(sl2, sl2), negm = make_float2(-m_use, -m_use);
+          float2 sum0 = make_float2(0.f, 0.f), sum1 = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int q = 0; q < kBN / 32; ++q) {
+            // a 32-column chunk outside every lane's [lo, hi) needs no exponentials
+            const bool need = __any_sync(0xffffffffu, lo < q * 32 + 32 && hi > q * 32);
+            if (need) {
+#pragma unroll
+              for (int c = 0; c < 32; c += 4) {
+                float2 e0 = ffma2(make_float2(S_(q * 32 + c), S_(q * 32 + c + 1)), sl2x2, negm);
+                float2 e1 = ffma2(make_float2(S_(q * 32 + c + 2), S_(q * 32 + c + 3)), sl2x2, negm);
+                e0 = make_float2(ex2(e0.x), ex2(e0.y));
+                e1 = make_float2(ex2(e1.x), ex2(e1.y));
+                sum0 = fadd2(sum0, e0);
+                sum1 = fadd2(sum1, e1);
+                pk[q * 16 + c / 2] = pack_bf16x2(e0.x, e0.y);
+                pk[q * 16 + c / 2 + 1] = pack_bf16x2(e1.x, e1.y);
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < 16; ++c) pk[q * 16 + c] = 0u;
+            }
+          }
+          const float2 s2 = fadd2(sum0, sum1);
+          tsum = s2.x + s2.y;
+        };
+        // a row with keys in this tile but no reference yet takes its max first
+        const bool no_ref = m_ref == -INFINITY && hi > lo;
+        if (__any_sync(0xffffffffu, no_ref)) {
+          const float mt = row_max();
+          if (no_ref) m_ref = mt;
         }
+        exps();
+        float fscale = 1.f;
+        bool grow = false;
+        if (__any_sync(0xffffffffu, !(tsum <= 65536.f))) {
+          const float mt = row_max();
+          grow = mt > m_ref;   // only rows whose max rose past the reference (a row's new keys
+                               // never lower it)
+          if (grow) {
+            fscale = ex2(m_ref - mt);   // brings this row's O and l to the new reference
+            l_run *= fscale;
+            m_ref = mt;
+          }
+          exps();
+        }
+        const bool rescale = j > 0 && __any_sync(0xffffffffu, grow);
 #undef S_
-        const float2 sum2 = fadd2(sum0, sum1);
-        l_run += sum2.x + sum2.y;
+        l_run += tsum;
         // P buffer g & 1 was last read by the PV of tile g - 2
         if (g >= 2 && !wait_pv(g - 2)) { ok = false; break; }
         tc_fence_after();
