@@ -32,6 +32,8 @@
 //              16-byte pieces into the segment each 8-column group belongs to,
 //              then tells the first CTA the accumulator is free
 // All waits are bounded; a give-up raises ATTAMBA_DEV_TIMEOUT.
+#include <mutex>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -50,6 +52,7 @@ constexpr uint32_t kBarOff = kStages * kStageBytes;
 constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;     // + barriers + alignment slack
 constexpr uint32_t kTmemCols = 512;                       // two 256-column accumulators
 constexpr uint64_t kWaitNs = 4000000000ull;
+constexpr int kMaxDevices = 64;
 
 struct Bars {
   uint64_t full[kStages];  // first CTA: both CTAs' operands of the stage have landed
@@ -294,26 +297,40 @@ cudaError_t launch_proj_gemm(const ProjArgs& a, cudaStream_t s) {
   if (!encode_2d(&tx, a.X, a.M, a.K, kBM) || !encode_2d(&tw, a.W, a.Nout, a.K, kBN / 2)) return cudaErrorNotSupported;
   cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(proj_gemm_kernel), (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  // as many CTA pairs as can be resident at once (a GPC with an odd number of free SMs leaves one out)
-  static int max_pairs = 0;
-  if (max_pairs == 0) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * (unsigned)(device_sm_count() / 2));
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, proj_gemm_kernel, &cfg) != cudaSuccess || n < 1) n = device_sm_count() / 2;
-    max_pairs = n;
+  // as many CTA pairs as can be resident at once (a GPC with an odd number of free SMs leaves one
+  // out), asked of the runtime once per device
+  static std::mutex mu;
+  static int max_pairs[kMaxDevices] = {};
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  int pairs_max;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (max_pairs[dev] == 0) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * (unsigned)(device_sm_count() / 2));
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = kSmemBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, proj_gemm_kernel, &cfg) != cudaSuccess || n < 1) {
+        cudaGetLastError();   // a failed query is not an error of this call
+        n = device_sm_count() / 2;
+      }
+      max_pairs[dev] = n;
+    }
+    pairs_max = max_pairs[dev];
   }
   const int64_t tiles = ((a.M + 2 * kBM - 1) / (2 * kBM)) * ((a.Nout + kBN - 1) / kBN);
-  const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
+  const int64_t pairs = tiles < pairs_max ? tiles : pairs_max;
   const int grid = (int)(2 * (pairs > 0 ? pairs : 1));
   proj_gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(tx, tw, a);
   return cudaGetLastError();

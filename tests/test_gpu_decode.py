@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import BF16_ATOL, f64, run_prefill
+from helpers import BF16_ATOL, BF16_HALF_ULP, assert_bf16_close, f64, run_prefill
 from oracle import decode as OD
 from ssm_compressed_chunked_b200 import attamba as A
 from ssm_compressed_chunked_b200 import workloads as W
@@ -82,6 +82,57 @@ def test_decode_workload_128_steps():
     p = cache.bpos[0, last].item()
     if p > end - 1 - cfg.L:
         assert torch.equal(cache.Kb[:, :, last], cache.Kr[:, :, p % cfg.L])
+
+
+def decode_rounding_bound(oc, b, q, o_ref, ctx, scale):
+    """First-order effect on the output of keys the GPU stored in bf16 while the oracle keeps them in
+    float64: the keys and values written during the decode (positions >= ctx; the synthetic cache
+    itself is bf16 on both sides).  Same rule as the prefill attention's: a change dv moves o by at most
+    max |dv|, a change dk moves a score by at most scale sum |q| |dk| and o by at most
+    max |v - o| times that.  Returns [H, dh]."""
+    t = oc.pos[b] - 1
+    lo = max(0, t - oc.L + 1)
+    ks, vs = [], []
+    for p, kk, vv in zip(oc.bpos[b], oc.Kb[b], oc.Vb[b]):
+        if ctx <= p < lo:
+            ks.append(kk)
+            vs.append(vv)
+    for p in range(max(lo, ctx), t + 1):
+        kk, vv = oc.ring[b][p]
+        ks.append(kk)
+        vs.append(vv)
+    if not ks:
+        return np.zeros_like(o_ref)
+    k = np.stack(ks)                                               # [j, H, dh]
+    v = np.stack(vs)
+    ds = scale * BF16_HALF_ULP * np.einsum("hd,jhd->jh", np.abs(q), np.abs(k)).max(axis=0)    # [H]
+    dv = BF16_HALF_ULP * np.abs(v).max(axis=0)                                                 # [H, dh]
+    spread = np.abs(v - o_ref[None]).max(axis=0)
+    return dv + spread * ds[:, None]
+
+
+@pytest.mark.parametrize("ctx,L,offset", [(16384, 64, 0), (5000, 40, 5)])
+def test_decode_many_splits(ctx, L, offset):
+    """Few (sequence, head) pairs over a long context: the step splits each key set many ways (16 at
+    ctx 16384), so splits start and end inside stages, one stage mixes boundary rows with ring rows
+    before and after the ring's wrap, and the last split holds the newest key."""
+    cfg = W.shrink(W.DECODE_CONFIG, B=1, H=2, D=128, ctx=ctx, L=L, offset=offset, steps=24, seed=31)
+    dec = W.make_decode(cfg)
+    g, cache = gpu_cache(dec)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    outs = run_steps(dec, g, cache, cfg.steps, status)
+    assert status.item() == 0
+    rows = [0]
+    oc = oracle_cache(dec, rows)
+    for s in range(cfg.steps):
+        sel = lambda t: f64(t[s][rows])
+        ro = oc.step(sel(dec["q"]), sel(dec["x"]), np.stack([f64(dec["dt_k"][s][rows]), f64(dec["dt_v"][s][rows])]),
+                     np.stack([f64(dec["bias_k"]), f64(dec["bias_v"])]), np.stack([f64(dec["A_k"]), f64(dec["A_v"])]),
+                     np.stack([f64(dec["B_k"][s][rows]), f64(dec["B_v"][s][rows])]),
+                     np.stack([f64(dec["C_k"][s][rows]), f64(dec["C_v"][s][rows])]), dec["scale"])
+        extra = decode_rounding_bound(oc, 0, f64(dec["q"][s][0]), ro[0], ctx, dec["scale"])
+        assert_bf16_close(f64(outs[s][rows])[0], ro[0], f"step {s}", extra=extra)
+    assert torch.all(cache.pos == ctx + cfg.steps)
 
 
 @pytest.mark.parametrize("P,offset,L,N", [(4, 0, 3, 16), (8, 3, 8, 16), (3, 1, 1, 16), (8, 3, 8, 32)])
