@@ -64,6 +64,30 @@ def test_attention_small(cfg):
     assert pf.status.item() == 0
 
 
+@pytest.mark.parametrize("qscale", [6.0, 40.0])
+def test_attention_wide_score_range(qscale):
+    """q scaled up so a row's scores spread over tens (6x) to hundreds (40x) of units of log2: later
+    tiles often hold a score far above the row's reference, so the kernel's row sum passes 2^16 or
+    overflows and it moves the reference, recomputes P and rescales O (stage-isolated check)."""
+    cfg = W.shrink(C2, B=2, n=520, D=128, H=2)
+    inp = W.make_layer(cfg)
+    inp["q"] = (inp["q"].float() * qscale).to(inp["q"].dtype)
+    pf = run_prefill(inp, cfg)
+    n, H, dh = cfg.n, cfg.H, cfg.dh
+    O = pf.O.view(cfg.B, n, H, dh)
+    lse = pf.lse.cpu().numpy()
+    K = pf.K.view(cfg.B, n, H, dh)
+    V = pf.V.view(cfg.B, n, H, dh)
+    for b in range(cfg.B):
+        st = np.asarray(inp["starts"][b])
+        ro, rl = oracle_attention_seq(f64(inp["q"][b]), f64(K[b]), f64(V[b]), st, n, cfg.L, cfg.mode, inp["scale"])
+        assert_close(cfg.dtype, f64(O[b]), ro, f"O (q x {qscale}) b={b}")
+        fin = np.isfinite(rl)
+        assert np.array_equal(np.isfinite(lse[b]), fin)
+        assert_close(cfg.dtype, lse[b][fin], rl[fin], f"lse (q x {qscale}) b={b}")
+    assert pf.status.item() == 0
+
+
 @pytest.mark.parametrize("cfg", [C1, C2, C3], ids=lambda c: c.name)
 def test_attention_full_size_sampled_rows(cfg):
     """Full-size configs in the bench's launch configuration; the oracle recomputes sampled query rows."""
