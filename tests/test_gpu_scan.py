@@ -101,3 +101,25 @@ def test_scan_kept_projection_inputs(cfg):
                                        f64(inp["A_" + name]), f64(inp["B_" + name][b]), f64(inp["C_" + name][b]),
                                        is_start)
             assert_close(cfg.dtype, f64(out[sl]), ref, f"{name} b={b}")
+
+
+@pytest.mark.parametrize("dtype_cfg", [W.shrink(W.LAYER_CONFIGS[0], B=1, n=96, D=64, H=1, P=8, offset=0),
+                                       W.shrink(W.LAYER_CONFIGS[2], B=1, n=96, D=64, H=1)],
+                         ids=["f32", "bf16"])
+def test_scan_softplus_regimes(dtype_cfg):
+    """dt spread over [-120, 40] so softplus(dt + bias) meets each regime of the kernel's evaluation:
+    the linear one above 20, the logarithm of 1 + e^z around 0, the series for small e^z, and steps
+    whose e^z underflows in fp32 (no decay and no input at all)."""
+    cfg = dtype_cfg
+    inp = W.make_layer(cfg)
+    gen = torch.Generator().manual_seed(77)
+    for k in ("dt_k", "dt_v"):
+        z = (torch.rand(inp[k].shape, generator=gen) * 160.0 - 120.0)
+        inp[k] = z.to(inp[k].dtype)
+    pf = run_prefill(inp, cfg)
+    K = pf.K.view(cfg.B, cfg.n, cfg.D)
+    V = pf.V.view(cfg.B, cfg.n, cfg.D)
+    rk, rv = oracle_scan_seq(inp, 0)
+    assert_close(cfg.dtype, f64(K[0]), rk, "K")
+    assert_close(cfg.dtype, f64(V[0]), rv, "V")
+    assert pf.status.item() == 0
