@@ -122,3 +122,20 @@ def test_value_one_gives_output_one():
     pf.attn_step(inp["q"].cuda(), inp["scale"])
     torch.cuda.synchronize()
     np.testing.assert_allclose(f64(pf.O), 1.0, atol=1e-2)
+
+
+@pytest.mark.parametrize("cfg", [W.shrink(C2, B=2, n=520, D=128, H=2), W.shrink(W.LAYER_CONFIGS[0], B=1, n=200)],
+                         ids=["bf16", "f32"])
+def test_attention_without_lse(cfg):
+    """The LSE output is optional: without it the same O comes out, bit for bit."""
+    from ssm_compressed_chunked_b200 import attamba as A
+    inp = W.make_layer(cfg)
+    pf = run_prefill(inp, cfg)
+    H, dh = cfg.H, cfg.dh
+    O2 = torch.full_like(pf.O, float("nan"))
+    q = inp["q"].to(pf.O.device).reshape(-1, H, dh)
+    A.chunk_attn_fwd(q, pf.K.view(-1, H, dh), pf.V.view(-1, H, dh), pf.Kc.view(-1, H, dh), pf.Vc.view(-1, H, dh),
+                     pf.index, inp["scale"], O2, None, pf.status)
+    torch.cuda.synchronize()
+    assert pf.status.item() == 0
+    assert torch.equal(O2, pf.O)
