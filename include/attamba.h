@@ -224,6 +224,12 @@ attamba_status_t attamba_cache_from_prefill(attamba_dtype_t dtype, const attamba
                                             const void* C_v, int32_t n0, int32_t* d_status,
                                             attamba_stream_t stream);
 
+/* Bytes of device memory a bf16 decode cache with the dimensions in `cache` takes (its
+ * pointers are not read): the arrays state, Kb, Vb, bpos, Kr, Vr, nb, pos in that order,
+ * each rounded up to 256 bytes, so one allocation of this size holds them all at
+ * 256-byte aligned offsets.  0 for a dimension out of range (B, H, N, L, cap < 1, dh != 64). */
+size_t attamba_cache_bytes(const attamba_cache_t* cache);
+
 /* Bytes of device workspace attamba_decode_step needs for this cache. */
 size_t attamba_decode_workspace_size(const attamba_cache_t* cache);
 

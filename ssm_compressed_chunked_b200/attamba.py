@@ -24,7 +24,7 @@ DEV_BAD_CHUNKS, DEV_CACHE_FULL, DEV_TIMEOUT = 0x1, 0x2, 0x4
 # every symbol include/attamba.h declares
 EXPORTS = ("attamba_version", "attamba_status_string", "attamba_last_error",
            "attamba_uniform_chunk_count", "attamba_chunk_index", "attamba_kv_ssm_scan",
-           "attamba_chunk_attn_fwd", "attamba_decode_workspace_size", "attamba_decode_step",
+           "attamba_chunk_attn_fwd", "attamba_cache_bytes", "attamba_decode_workspace_size", "attamba_decode_step",
            "attamba_decode_step_noalloc", "attamba_cache_from_prefill",
            "attamba_kv_ssm_scan_u", "attamba_proj_gemm")
 
@@ -80,6 +80,8 @@ def load():
     L.attamba_chunk_attn_fwd.restype = ctypes.c_int
     L.attamba_chunk_attn_fwd.argtypes = [ctypes.c_int, vp, vp, vp, vp, vp, ctypes.POINTER(IndexT),
                                          i32, i32, f32, vp, vp, vp, vp]
+    L.attamba_cache_bytes.restype = sz
+    L.attamba_cache_bytes.argtypes = [ctypes.POINTER(CacheT)]
     L.attamba_decode_workspace_size.restype = sz
     L.attamba_decode_workspace_size.argtypes = [ctypes.POINTER(CacheT)]
     L.attamba_decode_step.restype = ctypes.c_int
@@ -224,6 +226,14 @@ class Cache:
         return CacheT(self.state.data_ptr(), self.Kb.data_ptr(), self.Vb.data_ptr(), self.bpos.data_ptr(),
                       self.Kr.data_ptr(), self.Vr.data_ptr(), self.nb.data_ptr(), self.pos.data_ptr(),
                       self.B, self.H, self.dh, self.N, self.P, self.offset, self.L, self.cap)
+
+
+def cache_bytes(B, H, dh, N, L, cap):
+    """attamba_cache_bytes: device bytes of a bf16 decode cache with these dimensions (arrays at
+    256-byte aligned offsets: state, Kb, Vb, bpos, Kr, Vr, nb, pos)."""
+    c = CacheT()
+    c.B, c.H, c.dh, c.N, c.L, c.cap = int(B), int(H), int(dh), int(N), int(L), int(cap)
+    return int(load().attamba_cache_bytes(ctypes.byref(c)))
 
 
 def decode_workspace_size(cache):

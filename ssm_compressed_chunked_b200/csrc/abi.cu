@@ -177,6 +177,20 @@ attamba_status_t attamba_chunk_attn_fwd(attamba_dtype_t dtype, const void* q, co
   return e == cudaSuccess ? ATTAMBA_OK : cuda_fail(e, "attamba_chunk_attn_fwd");
 }
 
+size_t attamba_cache_bytes(const attamba_cache_t* cache) {
+  if (!cache || cache->B < 1 || cache->H < 1 || cache->N < 1 || cache->L < 1 || cache->cap < 1 || cache->dh != 64)
+    return 0;
+  const uint64_t B = (uint64_t)cache->B, H = (uint64_t)cache->H, dh = (uint64_t)cache->dh;
+  const uint64_t N = (uint64_t)cache->N, L = (uint64_t)cache->L, cap = (uint64_t)cache->cap;
+  auto up = [](uint64_t bytes) { return (bytes + 255) & ~uint64_t(255); };
+  const uint64_t bytes = up(2 * B * N * H * dh * 4)          // state [2, B, N, D] fp32
+                         + 2 * up(B * H * cap * dh * 2)     // Kb, Vb [B, H, cap, dh] bf16
+                         + up(B * cap * 4)                  // bpos [B, cap] int32
+                         + 2 * up(B * H * L * dh * 2)       // Kr, Vr [B, H, L, dh] bf16
+                         + 2 * up(B * 4);                   // nb, pos [B] int32
+  return (size_t)bytes;
+}
+
 size_t attamba_decode_workspace_size(const attamba_cache_t* cache) {
   if (!cache || cache->B < 1 || cache->H < 1 || cache->cap < 1 || cache->L < 1) return 0;
   return attamba::decode_workspace_bytes(*cache);

@@ -82,3 +82,28 @@ def test_cpu_tensors_are_refused():
     import torch
     with pytest.raises(A.AttambaError):
         A._ptr(torch.zeros(4), None, "x")
+
+
+@pytest.mark.parametrize("B,H,N,L,cap", [(1, 1, 16, 1, 1), (2, 16, 16, 64, 513), (3, 5, 32, 7, 33)])
+def test_cache_bytes_covers_every_cache_array(B, H, N, L, cap):
+    import torch
+    dh = 64
+    D = H * dh
+    arrays = [torch.empty(2, B, N, D, dtype=torch.float32, device="meta"),
+              torch.empty(B, H, cap, dh, dtype=torch.bfloat16, device="meta"),
+              torch.empty(B, H, cap, dh, dtype=torch.bfloat16, device="meta"),
+              torch.empty(B, cap, dtype=torch.int32, device="meta"),
+              torch.empty(B, H, L, dh, dtype=torch.bfloat16, device="meta"),
+              torch.empty(B, H, L, dh, dtype=torch.bfloat16, device="meta"),
+              torch.empty(B, dtype=torch.int32, device="meta"),
+              torch.empty(B, dtype=torch.int32, device="meta")]
+    off = 0
+    for t in arrays:
+        assert off % 256 == 0
+        off += -(-t.numel() * t.element_size() // 256) * 256
+    assert A.cache_bytes(B, H, dh, N, L, cap) == off
+    # degenerate dimensions give 0
+    assert A.cache_bytes(B, H, 32, N, L, cap) == 0
+    assert A.cache_bytes(0, H, dh, N, L, cap) == 0
+    assert A.cache_bytes(B, H, dh, N, 0, cap) == 0
+    assert A.cache_bytes(B, H, dh, N, L, 0) == 0
