@@ -650,6 +650,25 @@ def run_ours(args, ws, rank, local):
         roof["traffic"] = ncu_traffic("kv_ssm_scan_kernel" if dom == "kv_ssm_scan" else "chunk_index_kernel")
     roof["kernel"] = dom
     scan = kernels["kv_ssm_scan"]
+    # each kernel's binding bound: the slowest of its algorithmic bytes at the HBM copy rate, its
+    # exponentials at 16/clk/SM, its FMA-pipe work at 128 lanes/clk/SM (3 per scan exponential) and
+    # its tensor flops at the bf16 burst peak; the hot path's fraction is their sum over the step
+    fma_rate = 128 * 148 * 1.965e9
+    attn_bytes = T * D * 2 * 4 + 2 * nch * D * 2   # q, K, V read and O written once, chunk-end rows Kc, Vc
+    limits = {
+        "chunk_index": {"hbm": index_bytes / (hbm * 1e9)},
+        "kv_ssm_scan": {"hbm": scan_bytes / (hbm * 1e9), "exp": scan_exps / exp_peak, "fma": 3 * scan_exps / fma_rate},
+        "chunk_attn_fwd": {"hbm": attn_bytes / (hbm * 1e9), "exp": attn_flops / (4 * dh) / exp_peak,
+                           "tensor": attn_flops / (tf_burst * 1e12)},
+    }
+    hot = {}
+    for k, lim in limits.items():
+        b = max(lim, key=lim.get)
+        hot[k] = {"bound": b, "bound_us": round(lim[b] * 1e6, 2), "measured_us": round(kernels[k]["ms"] * 1e3, 2),
+                  "frac": round(lim[b] / (kernels[k]["ms"] * 1e-3), 4)}
+    sum_bound = sum(v["bound_us"] for v in hot.values())
+    hot_path = {"kernels": hot, "sum_bound_us": round(sum_bound, 2), "step_us": round(ms * 1e3, 2),
+                "frac": round(sum_bound / (ms * 1e3), 4)}
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -663,6 +682,7 @@ def run_ours(args, ws, rank, local):
                           "hbm_frac": scan["bytes"] / (scan["ms"] * 1e-3) / 1e9 / hbm},
         "attn_tensor": {"achieved_TFLOP_s": attn_flops / (mean[2] * 1e-3) / 1e12,
                         "frac_of_burst": attn_flops / (mean[2] * 1e-3) / 1e12 / tf_burst},
+        "hot_path_bound": hot_path,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 3 * args.steps,
         "clocks": clocks,

@@ -24,10 +24,15 @@
 //              pairs back into TMEM with one tcgen05.st
 // TMEM per CTA (256 columns): S in two buffers of 64, P in two of 32, O 64.
 // With S and P double-buffered the QK of tile g + 1 and the PV of tile g - 1
-// run while the softmax works on tile g; the softmax waits only for the PV
-// that last read the P buffer it is about to fill (tile g - 2).  Because the
-// four softmax warps can then drift up to two tiles apart, every barrier they
-// arrive on exists per buffer.  O accumulates in TMEM across an item's tiles;
+// run while the softmax works on tile g.  The one issuing thread orders the
+// MMAs PV(g - 2) before QK(g), and a tcgen05.commit arrives only once every
+// MMA that thread issued before it has completed, so two waits are implied
+// and not made: the softmax, having seen S(g), may refill P buffer g & 1 (its
+// last reader PV(g - 2) is done), and the issuer, having seen the P of tile
+// g - 2 arrive (each softmax thread arrives after its load of S(g - 2) has
+// completed), may overwrite S buffer g & 1 with QK(g).  Because the four
+// softmax warps can drift up to two tiles apart, every barrier they arrive on
+// exists per buffer.  O accumulates in TMEM across an item's tiles;
 // P = exp2(s - m_ref) against a per-row reference that only has to keep P
 // finite: it is the row max of the first tile where the row has keys, and it
 // moves to the current row max (P recomputed, O and l rescaled in TMEM) only
@@ -46,7 +51,10 @@
 // warps per SM sub-partition the tile's other instructions (about half of them
 // on the integer/logic pipe) and the barrier and TMEM latencies set the pace,
 // so each instruction taken out of the tile loop shows: the column mask and
-// the on-demand row max took 78.5 us to 70.6 us.  A third CTA does not fit (TMEM, shared memory); eight softmax
+// the on-demand row max took 78.5 us to 70.6 us, and dropping the two implied
+// waits to 66.5 us.  One thread issues a tcgen05.mma every ~90 cycles
+// (measured, N = 64 or 128 alike), so the eight MMAs of a tile keep the issuing
+// thread busy for ~720 of the ~1500 cycles a tile takes.  A third CTA does not fit (TMEM, shared memory); eight softmax
 // warps with the 16-lane TMEM shapes, 128-key tiles, and moving a share of the
 // exponentials to an FMA-pipe polynomial all measured slower.
 //
@@ -117,7 +125,6 @@ struct Bars {
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
   uint64_t s_full[2];    // QK of tile g done (tcgen05.commit)
-  uint64_t s_empty[2];   // every softmax thread has read S of tile g (128 arrivals)
   uint64_t p_full[2];    // every softmax thread has written P of tile g (128 arrivals)
   uint64_t pv_done[2];   // PV of tile g done (tcgen05.commit)
   uint64_t mma_done;
@@ -251,7 +258,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       mbar_init(&bars->q_full[b], 1);
       mbar_init(&bars->q_empty[b], 1);
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_empty[b], kBM);
       mbar_init(&bars->pv_done[b], 1);
       mbar_init(&bars->p_full[b], kBM);
     }
@@ -369,11 +375,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         for (int j = 0; j < it.NT; ++j, ++g) {
           const int st = g % kStages;
           if (!mbar_wait_bounded(&bars->kv_full[st], (g / kStages) & 1, abort_flag, kWaitNs)) { ok = false; break; }
-          // S buffer g & 1 was last read by the softmax for tile g - 2
-          if (g >= 2 && !mbar_wait_bounded(&bars->s_empty[g & 1], ((g - 2) >> 1) & 1, abort_flag, kWaitNs)) {
-            ok = false;
-            break;
-          }
+          // S buffer g & 1 was last read by the softmax for tile g - 2, whose P arrival (each thread
+          // makes it after its S load has completed) was waited for before PV(g - 2) was issued
           tc_fence_after();
           const uint32_t sk = smem_u32(smem + kKOff + st * kKVBytes);
 #pragma unroll
@@ -445,8 +448,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         tc_fence_after();
         uint32_t sr[kBN];
         tmem_ld64_sync(lane_base + kSCol + (g & 1) * kBN, &sr[0]);
-        tc_fence_before();
-        mbar_arrive(&bars->s_empty[g & 1]);
         // row max of the raw scores over the valid columns [lo, hi); masked columns become -inf in place
         if (lo != 0 || hi != kBN) {
           // the valid columns as two 32-bit masks; each column is then one bit test and one select
@@ -531,8 +532,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const bool rescale = j > 0 && __any_sync(0xffffffffu, grow);
 #undef S_
         l_run += tsum;
-        // P buffer g & 1 was last read by the PV of tile g - 2
-        if (g >= 2 && !wait_pv(g - 2)) { ok = false; break; }
+        // P buffer g & 1 was last read by the PV of tile g - 2: issued before S(g), so complete
+        // once the commit of S(g) arrived
         tc_fence_after();
         tmem_st32(lane_base + kPCol + (g & 1) * (kBN / 2), &pk[0]);
         if (rescale) {
