@@ -224,6 +224,13 @@ attamba_status_t attamba_cache_from_prefill(attamba_dtype_t dtype, const attamba
                                             const void* C_v, int32_t n0, int32_t* d_status,
                                             attamba_stream_t stream);
 
+/* Self-test of the device failure path (no counterpart in the method): one thread waits, with the
+ * same bounded wait every pipeline kernel uses, on a shared-memory barrier that nothing completes;
+ * after limit_ns nanoseconds (1e3 .. 1e9) it gives up, ORs ATTAMBA_DEV_TIMEOUT into *d_status
+ * (device memory, required) and returns, leaving the context usable.  No trap, no fault.
+ * ATTAMBA_ERR_INVALID_ARG for a null d_status or a limit out of range. */
+attamba_status_t attamba_selftest_wait_timeout(uint64_t limit_ns, int32_t* d_status, attamba_stream_t stream);
+
 /* Bytes of device memory a bf16 decode cache with the dimensions in `cache` takes (its
  * pointers are not read): the arrays state, Kb, Vb, bpos, Kr, Vr, nb, pos in that order,
  * each rounded up to 256 bytes, so one allocation of this size holds them all at

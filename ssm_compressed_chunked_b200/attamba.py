@@ -24,7 +24,7 @@ DEV_BAD_CHUNKS, DEV_CACHE_FULL, DEV_TIMEOUT = 0x1, 0x2, 0x4
 # every symbol include/attamba.h declares
 EXPORTS = ("attamba_version", "attamba_status_string", "attamba_last_error",
            "attamba_uniform_chunk_count", "attamba_chunk_index", "attamba_kv_ssm_scan",
-           "attamba_chunk_attn_fwd", "attamba_cache_bytes", "attamba_decode_workspace_size", "attamba_decode_step",
+           "attamba_chunk_attn_fwd", "attamba_cache_bytes", "attamba_selftest_wait_timeout", "attamba_decode_workspace_size", "attamba_decode_step",
            "attamba_decode_step_noalloc", "attamba_cache_from_prefill",
            "attamba_kv_ssm_scan_u", "attamba_proj_gemm")
 
@@ -80,6 +80,8 @@ def load():
     L.attamba_chunk_attn_fwd.restype = ctypes.c_int
     L.attamba_chunk_attn_fwd.argtypes = [ctypes.c_int, vp, vp, vp, vp, vp, ctypes.POINTER(IndexT),
                                          i32, i32, f32, vp, vp, vp, vp]
+    L.attamba_selftest_wait_timeout.restype = ctypes.c_int
+    L.attamba_selftest_wait_timeout.argtypes = [ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p]
     L.attamba_cache_bytes.restype = sz
     L.attamba_cache_bytes.argtypes = [ctypes.POINTER(CacheT)]
     L.attamba_decode_workspace_size.restype = sz
@@ -226,6 +228,13 @@ class Cache:
         return CacheT(self.state.data_ptr(), self.Kb.data_ptr(), self.Vb.data_ptr(), self.bpos.data_ptr(),
                       self.Kr.data_ptr(), self.Vr.data_ptr(), self.nb.data_ptr(), self.pos.data_ptr(),
                       self.B, self.H, self.dh, self.N, self.P, self.offset, self.L, self.cap)
+
+
+def selftest_wait_timeout(limit_ns, status, stream=None):
+    """attamba_selftest_wait_timeout: a bounded wait that nothing completes; sets DEV_TIMEOUT in status."""
+    L = load()
+    st = L.attamba_selftest_wait_timeout(int(limit_ns), _ptr(status, torch.int32, "status"), _stream(stream))
+    _check(st, "attamba_selftest_wait_timeout")
 
 
 def cache_bytes(B, H, dh, N, L, cap):

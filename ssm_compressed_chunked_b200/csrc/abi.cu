@@ -177,6 +177,12 @@ attamba_status_t attamba_chunk_attn_fwd(attamba_dtype_t dtype, const void* q, co
   return e == cudaSuccess ? ATTAMBA_OK : cuda_fail(e, "attamba_chunk_attn_fwd");
 }
 
+attamba_status_t attamba_selftest_wait_timeout(uint64_t limit_ns, int32_t* d_status, attamba_stream_t stream) {
+  if (!d_status || limit_ns < 1000 || limit_ns > 1000000000ull) return ATTAMBA_ERR_INVALID_ARG;
+  const cudaError_t e = attamba::launch_wait_selftest(limit_ns, d_status, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTAMBA_OK : cuda_fail(e, "attamba_selftest_wait_timeout");
+}
+
 size_t attamba_cache_bytes(const attamba_cache_t* cache) {
   if (!cache || cache->B < 1 || cache->H < 1 || cache->N < 1 || cache->L < 1 || cache->cap < 1 || cache->dh != 64)
     return 0;

@@ -3,6 +3,7 @@
 // kernel's dynamic shared-memory limit has been raised on the device.
 #include <mutex>
 
+#include "common.cuh"
 #include "launch.h"
 
 namespace attamba {
@@ -42,6 +43,27 @@ cudaError_t raise_smem_limit(const void* kernel, int bytes) {
     }
   }
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+namespace {
+// The give-up path every pipeline wait has, exercised on purpose: nothing ever arrives on `bar`, so
+// the bounded wait runs out after limit_ns and the status bit is raised; the kernel then returns.
+__global__ void wait_selftest_kernel(uint64_t limit_ns, int32_t* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0, &abort_flag, limit_ns)) raise_status(status, ATTAMBA_DEV_TIMEOUT);
+}
+}  // namespace
+
+cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t* status, cudaStream_t s) {
+  wait_selftest_kernel<<<1, 32, 0, s>>>(limit_ns, status);
+  return cudaGetLastError();
 }
 
 }  // namespace attamba

@@ -112,4 +112,7 @@ struct HandoffArgs {
 int32_t handoff_boundaries(int32_t n0, int32_t P, int32_t offset);
 cudaError_t launch_cache_from_prefill(const HandoffArgs& a, cudaStream_t s);
 
+// one CTA whose thread waits, with the pipelines' bounded wait, on a barrier that nothing completes
+cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t* status, cudaStream_t s);
+
 }  // namespace attamba

@@ -76,6 +76,10 @@ def test_invalid_arguments_are_rejected_on_the_host():
     assert lib.attamba_cache_from_prefill(1, ctypes.byref(c), *args, 0, None, None) == A.ERR_INVALID_ARG
     assert lib.attamba_cache_from_prefill(1, ctypes.byref(c), *args, 64, None, None) == A.ERR_INVALID_ARG
     assert b"exceed cap" in lib.attamba_last_error()
+    # wait self-test: status word required, limit within [1 us, 1 s]
+    assert lib.attamba_selftest_wait_timeout(1000000, None, None) == A.ERR_INVALID_ARG
+    assert lib.attamba_selftest_wait_timeout(999, fake, None) == A.ERR_INVALID_ARG
+    assert lib.attamba_selftest_wait_timeout(1000000001, fake, None) == A.ERR_INVALID_ARG
 
 
 def test_cpu_tensors_are_refused():
