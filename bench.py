@@ -36,7 +36,7 @@ from ssm_compressed_chunked_b200 import workloads as W  # noqa: E402
 
 METRIC = "Attamba layer fwd tokens/s at n=4096,P=8,L=64 bf16"
 UNIT = "tokens/s"
-CFG = W.LAYER_CONFIGS[2]
+CFG = W.BF16_TEST_P8_L64
 L2_FLUSH_BYTES = 256 << 20
 
 

@@ -67,6 +67,8 @@ LAYER_CONFIGS = [
     LayerConfig("bf16_test_P8_L64", 4, 4096, 1024, 16, 64, 16, 8, 0, 64, "test", "bf16", 2),
     LayerConfig("bf16_varlen_train", 4, 8192, 1024, 16, 64, 16, 0, 0, 32, "train", "bf16", 3, (2, 16)),
 ]
+# the same workloads by name
+TINY_F32_TRAIN, BF16_TRAIN_CYCLIC, BF16_TEST_P8_L64, BF16_VARLEN_TRAIN = LAYER_CONFIGS
 DECODE_CONFIG = DecodeConfig("bf16_decode", 32, 16384, 2048, 32, 64, 16, 8, 0, 64, 128, 4)
 
 

@@ -16,10 +16,10 @@ from ssm_compressed_chunked_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
 
-C1, C2, C3 = W.LAYER_CONFIGS[1], W.LAYER_CONFIGS[2], W.LAYER_CONFIGS[3]
+C1, C2, C3 = W.BF16_TRAIN_CYCLIC, W.BF16_TEST_P8_L64, W.BF16_VARLEN_TRAIN
 SMALL = [
-    W.LAYER_CONFIGS[0],                                                    # fp32, full size
-    W.shrink(W.LAYER_CONFIGS[0], B=2, n=200, P=8, offset=3, L=5, mode="test"),   # fp32 M_test
+    W.TINY_F32_TRAIN,                                                    # fp32, full size
+    W.shrink(W.TINY_F32_TRAIN, B=2, n=200, P=8, offset=3, L=5, mode="test"),   # fp32 M_test
     W.shrink(C1, B=2, n=300, D=128, H=2),                                  # M_train, offset 3, L 4, ragged
     W.shrink(C2, B=2, n=520, D=128, H=2),                                  # M_test P 8 L 64, 5 tiles
     W.shrink(C3, B=2, n=387, D=128, H=2),                                  # variable chunks
@@ -124,7 +124,7 @@ def test_value_one_gives_output_one():
     np.testing.assert_allclose(f64(pf.O), 1.0, atol=1e-2)
 
 
-@pytest.mark.parametrize("cfg", [W.shrink(C2, B=2, n=520, D=128, H=2), W.shrink(W.LAYER_CONFIGS[0], B=1, n=200)],
+@pytest.mark.parametrize("cfg", [W.shrink(C2, B=2, n=520, D=128, H=2), W.shrink(W.TINY_F32_TRAIN, B=1, n=200)],
                          ids=["bf16", "f32"])
 def test_attention_without_lse(cfg):
     """The LSE output is optional: without it the same O comes out, bit for bit."""

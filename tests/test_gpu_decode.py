@@ -139,7 +139,7 @@ def test_decode_many_splits(ctx, L, offset):
 def test_decode_from_empty_cache_equals_test_mask_prefill(P, offset, L, N):
     """Decoding n tokens one by one from an empty cache reproduces the M_test prefill (GPU vs GPU and vs oracle)."""
     B, n, H, dh = 2, 150, 2, 64
-    cfg = W.shrink(W.LAYER_CONFIGS[2], B=B, n=n, D=H * dh, H=H, P=P, offset=offset, L=L, mode="test", N=N)
+    cfg = W.shrink(W.BF16_TEST_P8_L64, B=B, n=n, D=H * dh, H=H, P=P, offset=offset, L=L, mode="test", N=N)
     inp = W.make_layer(cfg)
     pf = run_prefill(inp, cfg)
     cap = n // P + 2

@@ -22,7 +22,7 @@ def test_bounded_wait_gives_up_and_reports():
     assert elapsed < 2.0, elapsed   # the wait ended on its limit, far below the pipelines' 4 s
 
     # the context is still usable: a prefill chunk index right after matches the uniform layout
-    cfg = W.shrink(W.LAYER_CONFIGS[2], B=2, n=300, D=128, H=2)
+    cfg = W.shrink(W.BF16_TEST_P8_L64, B=2, n=300, D=128, H=2)
     inp = W.make_layer(cfg)
     nch = layer.n_chunks_of(cfg, inp["cu"])
     pf = layer.Prefill(cfg.B, cfg.n, cfg.D, cfg.H, cfg.dh, cfg.N, nch, torch.bfloat16)

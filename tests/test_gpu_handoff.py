@@ -38,7 +38,7 @@ def test_cache_from_prefill_matches_oracle_and_continues_the_prefill(P, offset, 
     B, H, dh, m = 2, 2, 64, 24
     n = n0 + m
     D = H * dh
-    cfg = W.shrink(W.LAYER_CONFIGS[2], B=B, n=n, D=D, H=H, P=P, offset=offset, L=L, mode="test", N=N)
+    cfg = W.shrink(W.BF16_TEST_P8_L64, B=B, n=n, D=D, H=H, P=P, offset=offset, L=L, mode="test", N=N)
     inp = W.make_layer(cfg)
     pf = run_prefill(inp, cfg)                      # M_test prefill over all n positions (reference rows)
     g = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}

@@ -70,9 +70,8 @@ def test_random_sweep():
         _check(starts, n, L, mode_s, idx, cu)
 
 
-@pytest.mark.parametrize("ci", range(4))
-def test_configs(ci):
-    cfg = W.LAYER_CONFIGS[ci]
+@pytest.mark.parametrize("cfg", W.LAYER_CONFIGS, ids=lambda c: c.name)
+def test_configs(cfg):
     gen = torch.Generator().manual_seed(cfg.seed)
     starts = W.chunk_starts(cfg, gen) if cfg.varlen is not None else \
         [W._uniform_starts(cfg.n, cfg.P, cfg.offset)] * cfg.B

@@ -11,16 +11,16 @@ from ssm_compressed_chunked_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 SMALL = [
-    W.LAYER_CONFIGS[0],                                                   # fp32, full size
-    W.shrink(W.LAYER_CONFIGS[1], B=2, n=300, D=128, H=2),                 # cyclic offset 3, ragged n
-    W.shrink(W.LAYER_CONFIGS[2], B=2, n=333, D=192, H=3),                 # P = 8
-    W.shrink(W.LAYER_CONFIGS[3], B=3, n=257, D=128, H=2),                 # variable chunks
-    W.shrink(W.LAYER_CONFIGS[1], B=1, n=64, D=64, H=1, P=1, offset=0),   # P = 1
-    W.shrink(W.LAYER_CONFIGS[1], B=2, n=50, D=64, H=1, P=64, offset=0),  # one chunk per sequence
-    W.shrink(W.LAYER_CONFIGS[0], B=2, n=77, D=64, H=1, P=16, offset=5),   # fp32 cyclic
-    W.shrink(W.LAYER_CONFIGS[2], B=2, n=200, D=128, H=2, N=32),           # state size 32 (the pages' default)
-    W.shrink(W.LAYER_CONFIGS[3], B=2, n=150, D=64, H=1, N=32),            # N = 32, variable chunks
-    W.shrink(W.LAYER_CONFIGS[0], B=1, n=96, D=64, H=1, N=32, offset=2),   # fp32, N = 32
+    W.TINY_F32_TRAIN,                                                   # fp32, full size
+    W.shrink(W.BF16_TRAIN_CYCLIC, B=2, n=300, D=128, H=2),                 # cyclic offset 3, ragged n
+    W.shrink(W.BF16_TEST_P8_L64, B=2, n=333, D=192, H=3),                 # P = 8
+    W.shrink(W.BF16_VARLEN_TRAIN, B=3, n=257, D=128, H=2),                 # variable chunks
+    W.shrink(W.BF16_TRAIN_CYCLIC, B=1, n=64, D=64, H=1, P=1, offset=0),   # P = 1
+    W.shrink(W.BF16_TRAIN_CYCLIC, B=2, n=50, D=64, H=1, P=64, offset=0),  # one chunk per sequence
+    W.shrink(W.TINY_F32_TRAIN, B=2, n=77, D=64, H=1, P=16, offset=5),   # fp32 cyclic
+    W.shrink(W.BF16_TEST_P8_L64, B=2, n=200, D=128, H=2, N=32),           # state size 32 (the pages' default)
+    W.shrink(W.BF16_VARLEN_TRAIN, B=2, n=150, D=64, H=1, N=32),            # N = 32, variable chunks
+    W.shrink(W.TINY_F32_TRAIN, B=1, n=96, D=64, H=1, N=32, offset=2),   # fp32, N = 32
 ]
 
 
@@ -41,10 +41,9 @@ def test_scan_small(cfg):
     assert pf.status.item() == 0
 
 
-@pytest.mark.parametrize("ci", [1, 2, 3])
-def test_scan_full_size_sampled_chunks(ci):
-    """Configs at full size, in the launch the bench times; the oracle recomputes sampled chunks."""
-    cfg = W.LAYER_CONFIGS[ci]
+@pytest.mark.parametrize("cfg", [W.BF16_TRAIN_CYCLIC, W.BF16_TEST_P8_L64, W.BF16_VARLEN_TRAIN], ids=lambda c: c.name)
+def test_scan_full_size_sampled_chunks(cfg):
+    """The workloads at full size, in the launch the bench times; the oracle recomputes sampled chunks."""
     inp = W.make_layer(cfg)
     pf = run_prefill(inp, cfg)
     K = pf.K.view(cfg.B, cfg.n, cfg.D)
@@ -61,8 +60,8 @@ def test_scan_full_size_sampled_chunks(ci):
     assert pf.status.item() == 0
 
 
-@pytest.mark.parametrize("cfg", [W.shrink(W.LAYER_CONFIGS[1], B=2, n=300, D=128, H=2),
-                                 W.shrink(W.LAYER_CONFIGS[0], B=2, n=77, D=64, H=1, P=16, offset=5)],
+@pytest.mark.parametrize("cfg", [W.shrink(W.BF16_TRAIN_CYCLIC, B=2, n=300, D=128, H=2),
+                                 W.shrink(W.TINY_F32_TRAIN, B=2, n=77, D=64, H=1, P=16, offset=5)],
                          ids=lambda c: f"{c.name}-n{c.n}-D{c.D}")
 def test_scan_kept_projection_inputs(cfg):
     """attamba_kv_ssm_scan_u: the keys SSM reads u_k = x W_K, the values SSM u_v = x W_V (the
@@ -103,8 +102,8 @@ def test_scan_kept_projection_inputs(cfg):
             assert_close(cfg.dtype, f64(out[sl]), ref, f"{name} b={b}")
 
 
-@pytest.mark.parametrize("dtype_cfg", [W.shrink(W.LAYER_CONFIGS[0], B=1, n=96, D=64, H=1, P=8, offset=0),
-                                       W.shrink(W.LAYER_CONFIGS[2], B=1, n=96, D=64, H=1)],
+@pytest.mark.parametrize("dtype_cfg", [W.shrink(W.TINY_F32_TRAIN, B=1, n=96, D=64, H=1, P=8, offset=0),
+                                       W.shrink(W.BF16_TEST_P8_L64, B=1, n=96, D=64, H=1)],
                          ids=["f32", "bf16"])
 def test_scan_softplus_regimes(dtype_cfg):
     """dt spread over [-120, 40] so softplus(dt + bias) meets each regime of the kernel's evaluation:
