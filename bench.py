@@ -505,118 +505,6 @@ def run_ours(args, ws, rank, local):
     assert torch.equal(o_e2e, pf.O.cpu()), "end-to-end output differs from the resident-input step"
 
     assert pf.status.item() == 0, f"device status {pf.status.item()}"
-    return rows
-
-
-# ------------------------------------------------------------------ CUDA path
-def run_ours(args, ws, rank, local):
-    from ssm_compressed_chunked_b200 import attamba as A, layer
-
-    dev = torch.device("cuda", local)
-    cfg = rank_config(CFG, ws, rank)
-    inp = W.make_layer(cfg)
-    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
-    nch = layer.n_chunks_of(cfg, inp["cu"])
-    pf = layer.Prefill(cfg.B, cfg.n, cfg.D, cfg.H, cfg.dh, cfg.N, nch, torch.bfloat16, dev)
-    mode = layer.mode_code(cfg.mode)
-    stream = torch.cuda.current_stream(dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-
-    def step(events=None, src=None):
-        """One step: chunk_index, kv_ssm_scan, chunk_attn_fwd on the inputs `src` (default: the
-        resident set).  Two events bracket the step; four also split it per call (an event between two
-        calls keeps the second call's launch from overlapping the first call's tail, so the split sums
-        to a little more than the step)."""
-        src = g if src is None else src
-        if events:
-            events[0].record(stream)
-        pf.index_step(None, cfg.P, cfg.offset, cfg.L, mode)
-        if events and len(events) == 4:
-            events[1].record(stream)
-        pf.scan_step(src["x"], src["dt_k"], src["dt_v"], g["bias_k"], g["bias_v"], g["A_k"], g["A_v"], src["B_k"],
-                     src["C_k"], src["B_v"], src["C_v"])
-        if events and len(events) == 4:
-            events[2].record(stream)
-        pf.attn_step(src["q"], inp["scale"])
-        if events:
-            events[-1].record(stream)
-
-    sampler = ClockSampler(local) if rank == 0 else None
-    t_w = time.perf_counter()
-    nw = 0
-    while nw < max(3, args.warmup) or (time.perf_counter() - t_w) * 1e3 < args.min_warmup_ms:
-        flush.fill_(1)
-        step()
-        nw += 1
-        if nw % 16 == 0:
-            torch.cuda.synchronize()
-    torch.cuda.synchronize()
-
-    # algorithmic work of one step
-    T, D, N, H, dh = cfg.B * cfg.n, cfg.D, cfg.N, cfg.H, cfg.dh
-    ls = pf.index.ls.cpu().numpy().astype(np.int64)
-    nbb = pf.index.nbb.cpu().numpy().astype(np.int64)
-    i = np.tile(np.arange(cfg.n), cfg.B)
-    keys = int((nbb + np.maximum(0, i - ls + 1)).sum())
-    attn_flops = 4.0 * dh * H * keys
-    scan_bytes = T * (5 * D * 2 + 4 * N * 2) + 2 * nch * D * 2
-    scan_exps = 2.0 * T * D * N
-    index_bytes = T * 8 + nch * 8
-
-    # timed region: K steps, each bracketed by two events on the launching stream (the L2 flush
-    # between steps lies outside them)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    barrier(ws)
-    torch.cuda.synchronize()
-    if sampler:
-        sampler.mark()
-    for k in range(args.steps):
-        flush.fill_(k & 0xFF)
-        step(evs[k])
-    torch.cuda.synchronize()
-    barrier(ws)
-    clocks = sampler.stop() if sampler else None
-    step_ms = np.array([evs[k][0].elapsed_time(evs[k][1]) for k in range(args.steps)])
-    ms = max_over_ranks(float(step_ms.mean()), ws)
-    value = job_throughput(ws, T, ms)
-
-    # per-call split (roofline of each kernel): the same K steps again with events between the calls
-    evk = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    for k in range(args.steps):
-        flush.fill_(k & 0xFF)
-        step(evk[k])
-    torch.cuda.synchronize()
-    per = np.array([[evk[k][j].elapsed_time(evk[k][j + 1]) for j in range(3)] for k in range(args.steps)])  # ms
-
-    # end to end through the public API with host buffers: pinned H2D of the step's activations,
-    # the three calls, D2H of the output
-    names = ["x", "q", "dt_k", "dt_v", "B_k", "C_k", "B_v", "C_v"]
-    host = {k: inp[k].pin_memory() for k in names}
-    h_out = torch.empty(pf.O.shape, dtype=pf.O.dtype).pin_memory()
-    h2d = sum(host[k].numel() * host[k].element_size() for k in names)
-    d2h = h_out.numel() * h_out.element_size()
-    e2e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-
-    def e2e_step():
-        for k in names:
-            g[k].copy_(host[k], non_blocking=True)
-        step()
-        h_out.copy_(pf.O, non_blocking=True)
-
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    e2e_steps = max(3, min(args.steps, 10))
-    barrier(ws)
-    e2e_ev[0].record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e2e_ev[1].record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e2e_ev[0].elapsed_time(e2e_ev[1]) / e2e_steps, ws)
-    e2e_value = job_throughput(ws, T, e2e_ms)
-
-    assert pf.status.item() == 0, f"device status {pf.status.item()}"
     if rank != 0:
         return
 

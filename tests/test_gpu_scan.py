@@ -48,7 +48,7 @@ def test_scan_full_size_sampled_chunks(cfg):
     pf = run_prefill(inp, cfg)
     K = pf.K.view(cfg.B, cfg.n, cfg.D)
     V = pf.V.view(cfg.B, cfg.n, cfg.D)
-    rng = np.random.default_rng(ci)
+    rng = np.random.default_rng(cfg.seed)
     for b in (0, cfg.B - 1):
         st = list(inp["starts"][b]) + [cfg.n]
         picks = {0, len(st) - 2} | set(rng.integers(0, len(st) - 1, size=4).tolist())
