@@ -288,7 +288,9 @@ def decode_bench(dev, reps=3):
 def next_rows_bench(cfg, g, inp, pf, nch, dev, flush, scan_exps, reps=10):
     """The rows built after the hot path, timed on the bench workload's shapes (L2 flushed before each
     launch, median of CUDA-event times on the launching stream): the projection GEMMs, the kept-projection
-    scan (one input per SSM), the scan at the pages' state size N = 32, and the prefill -> decode handoff."""
+    scan (one input per SSM), the scan at the pages' state size N = 32, the prefill -> decode handoff, and
+    the whole layer with its projections (device-resident x, then x in and y out through pinned host
+    memory)."""
     import math
     from ssm_compressed_chunked_b200 import attamba as A
 
@@ -369,6 +371,59 @@ def next_rows_bench(cfg, g, inp, pf, nch, dev, flush, scan_exps, reps=10):
         "output": {"us": ms_o * 1e3, "TFLOP_s": fl_o / (ms_o * 1e-3) / 1e12,
                    "frac_of_bf16_burst": fl_o / (ms_o * 1e-3) / 1e12 / tf_burst},
         "traffic_inputs": ncu_traffic("proj_gemm_kernel")}
+
+    # the layer with its projections: x -> the seven input projections (one GEMM) -> chunk_index,
+    # kv_ssm_scan, chunk_attn_fwd -> W_O.  Timed with x resident, then end to end with x copied in from
+    # pinned host memory and y copied back every step (copies on streams of their own, two x buffers,
+    # so step k + 1's x crosses PCIe while step k computes)
+    from ssm_compressed_chunked_b200 import layer
+    mode = layer.mode_code(cfg.mode)
+    q_, dtk_, dtv_, bk_, ck_, bv_, cv_ = [o for o, _ in outs]
+
+    def layer_fwd(xs):
+        A.proj_gemm(xs, W_in, outs, pf.status)
+        pf.index_step(None, cfg.P, cfg.offset, cfg.L, mode)
+        pf.scan_step(xs, dtk_, dtv_, g["bias_k"], g["bias_v"], g["A_k"], g["A_v"], bk_, ck_, bv_, cv_)
+        pf.attn_step(q_.view(T, H, dh), inp["scale"])
+        A.proj_gemm(pf.O.view(T, H * dh), W_O, [(y, 0)], pf.status)
+
+    ms_layer = timed(lambda: layer_fwd(flat(g["x"])))
+    h_x = inp["x"].reshape(T, D).pin_memory()
+    h_y = torch.empty(T, D, dtype=bf).pin_memory()
+    xs = [flat(g["x"]), torch.empty_like(flat(g["x"]))]
+    cp_in, cp_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def layer_e2e(n_steps):
+        ev_comp = [torch.cuda.Event() for _ in range(n_steps)]
+        ev_out = [torch.cuda.Event() for _ in range(n_steps)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(cp_in)
+        for k in range(n_steps):
+            if k >= 2:
+                cp_in.wait_event(ev_comp[k - 2])
+            with torch.cuda.stream(cp_in):
+                xs[k & 1].copy_(h_x, non_blocking=True)
+            ev_in = torch.cuda.Event()
+            ev_in.record(cp_in)
+            stream.wait_event(ev_in)
+            if k >= 1:
+                stream.wait_event(ev_out[k - 1])
+            layer_fwd(xs[k & 1])
+            ev_comp[k].record(stream)
+            cp_out.wait_event(ev_comp[k])
+            with torch.cuda.stream(cp_out):
+                h_y.copy_(y, non_blocking=True)
+            ev_out[k].record(cp_out)
+        t1.record(cp_out)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1) / n_steps
+
+    layer_e2e(2)
+    ms_e2e = layer_e2e(reps)
+    rows["layer_incl_projections"] = {
+        "us": ms_layer * 1e3, "tokens_per_s": T / (ms_layer * 1e-3),
+        "e2e_tokens_per_s": T / (ms_e2e * 1e-3), "h2d_bytes_per_step": T * D * 2, "d2h_bytes_per_step": T * D * 2,
+        "note": "x in, y = O W_O out; random-init projection weights of the workload's shapes"}
     assert pf.status.item() == 0, f"device status {pf.status.item()}"
     return rows
 
