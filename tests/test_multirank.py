@@ -47,3 +47,22 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
     import bench
     bench.run_reference(argparse.Namespace(steps=1, warmup=0), 2, 1)   # rank 1: no work, no output
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_prints_the_contract_line(capsys):
+    import argparse
+    import json
+    import bench
+    bench.run_reference(argparse.Namespace(steps=1, warmup=0), 1, 0)
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
+    assert d["higher_is_better"] is True and d["value"] > 0 and d["steps"] == 1
+    assert d["config"]["workload"] == bench.CFG.name
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
