@@ -24,7 +24,7 @@
 //
 // The work is one exponential per (token, channel, state, SSM): 2 T D N of them
 // against 10 D bytes per token, so the multi-function unit (16 ex2 per clock
-// per SM), not HBM, sets the pace; on the bench workload it is about 78% busy.
+// per SM), not HBM, sets the pace; on the bench workload it is about 80% busy.
 // An FMA-pipe alternative is compiled in for bf16 outputs but off by default
 // (ATTAMBA_SCAN_POLY_PAIRS = 0): kPolyPairs of the N/2 state pairs would take
 // 2^x = 2^j * 2^f with j = round(x) (added to the exponent field) and 2^f from a
