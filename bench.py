@@ -58,7 +58,7 @@ def config_block(cfg, extra=None):
 
 
 class ClockSampler:
-    """SM clock and clock-event (throttle) reasons sampled through NVML every ~2 ms in a thread.
+    """SM clock and clock-event (throttle) reasons sampled through NVML every ~0.5 ms in a thread.
 
     mark() opens the window whose samples are reported (the timed region)."""
 
@@ -95,7 +95,7 @@ class ClockSampler:
                 self.samples.append((time.perf_counter(), mhz, rs))
             except Exception:
                 pass
-            time.sleep(0.002)
+            time.sleep(0.0005)
 
     def mark(self):
         self.t_mark = time.perf_counter()
@@ -106,13 +106,13 @@ class ClockSampler:
         self.stop_evt.set()
         self.th.join(timeout=2)
         win = [x for x in self.samples if self.t_mark is None or x[0] >= self.t_mark]
-        if len(win) < 3:  # a very short timed region: widen to the last 0.5 s before it
+        if len(win) < 8:  # a very short timed region: widen to the last 0.5 s before it
             win = [x for x in self.samples if self.t_mark is None or x[0] >= self.t_mark - 0.5]
         if not win:
             return None
         reasons = sorted(k for k, bit in self.REASONS.items() if any(r & bit for _, _, r in win))
         return {"sm_mhz": statistics.median(m for _, m, _ in win), "sm_max_mhz": self.max_mhz,
-                "reasons": reasons, "samples": len(win), "source": "NVML, 2 ms period"}
+                "reasons": reasons, "samples": len(win), "source": "NVML, 0.5 ms period"}
 
 
 def source_sha(files):
