@@ -8,13 +8,18 @@ bf16): chunk index -> KV-SSM scan (K and V) -> chunk-masked attention, three
 C-ABI calls on inputs already resident in HBM.  L2 is flushed between steps
 (a 256 MiB write, outside the per-step events).  Each rank runs its own batch
 (weak scaling, no collective on the data path); the time is the max over ranks.
+``--gpus N`` with N > 1 runs one rank per GPU: started without a launcher, the
+script relaunches itself under torch.distributed.run with N processes on this
+node (rendezvous on 127.0.0.1); under a launcher, WORLD_SIZE must equal N.
 Each timed step is bracketed by two CUDA events on the launching stream (the
 scan and the attention are programmatic dependent launches, so nothing is
 recorded between the calls); a second pass of the same steps with events
 between the calls gives each kernel's time for the roofline.
 
 --impl reference times the CPU oracle (float64 numpy, test infrastructure) on
-this host's cores on a bounded sample of the same workload.
+this host's cores: each step is one head of sequence 0 of the same workload at
+its full length (both scans over that head's channels and its dense n x n
+attention), the heads taken in turn.
 """
 
 import argparse
@@ -175,21 +180,26 @@ def barrier(ws):
 
 
 # ------------------------------------------------------------------ CPU oracle (reference arm / baseline)
-def oracle_sample(inp, n_tok):
-    """The oracle on sequence 0 truncated to n_tok tokens, all heads: scan K/V + dense M_test attention."""
+def oracle_sample(inp, b=0, heads=None):
+    """The oracle on the whole of sequence b (all n tokens) for the heads ``heads`` (None: all):
+    the float64 scans of K and V over those heads' channels (channels are independent) and the dense
+    n x n M_test softmax attention of those heads."""
     from oracle import attention as OA, chunks as OC, mask as OM, ssm as OS
     cfg = inp["cfg"]
+    n, dh = cfg.n, cfg.dh
+    heads = list(range(cfg.H)) if heads is None else list(heads)
+    ch = np.concatenate([np.arange(h * dh, (h + 1) * dh) for h in heads])
     f = lambda t: t.detach().to(torch.float64).numpy()
-    st = OC.uniform_starts(n_tok, cfg.P, cfg.offset)
-    is_start = OC.is_start_mask(st, n_tok)
-    sl = slice(0, n_tok)
-    K, _ = OS.selective_scan(f(inp["x"][0, sl]), f(inp["dt_k"][0, sl]), f(inp["bias_k"]), f(inp["A_k"]),
-                             f(inp["B_k"][0, sl]), f(inp["C_k"][0, sl]), is_start)
-    V, _ = OS.selective_scan(f(inp["x"][0, sl]), f(inp["dt_v"][0, sl]), f(inp["bias_v"]), f(inp["A_v"]),
-                             f(inp["B_v"][0, sl]), f(inp["C_v"][0, sl]), is_start)
-    M = OM.dense_mask(n_tok, st, cfg.L, cfg.mode)
-    OA.masked_attention(f(inp["q"][0, sl]), K.reshape(n_tok, cfg.H, cfg.dh), V.reshape(n_tok, cfg.H, cfg.dh), M,
-                        inp["scale"])
+    st = OC.uniform_starts(n, cfg.P, cfg.offset)
+    is_start = OC.is_start_mask(st, n)
+    x = f(inp["x"][b])[:, ch]
+    K, _ = OS.selective_scan(x, f(inp["dt_k"][b])[:, ch], f(inp["bias_k"])[ch], f(inp["A_k"])[ch],
+                             f(inp["B_k"][b]), f(inp["C_k"][b]), is_start)
+    V, _ = OS.selective_scan(x, f(inp["dt_v"][b])[:, ch], f(inp["bias_v"])[ch], f(inp["A_v"])[ch],
+                             f(inp["B_v"][b]), f(inp["C_v"][b]), is_start)
+    M = OM.dense_mask(n, st, cfg.L, cfg.mode)
+    hn = len(heads)
+    OA.masked_attention(f(inp["q"][b])[:, heads], K.reshape(n, hn, dh), V.reshape(n, hn, dh), M, inp["scale"])
 
 
 def cpu_cores():
@@ -200,54 +210,94 @@ def cpu_cores():
 
 
 def run_reference(args, ws, rank):
+    """Each step is one head of sequence 0 at its full length (n tokens: that head's channels of
+    both scans and its dense n x n attention), the heads taken in turn; a step counts n / H tokens."""
     if rank != 0:
         return
     inp = W.make_layer(CFG)
-    n_tok = 1024
-    oracle_sample(inp, 256)  # import / first-touch
-    for _ in range(args.warmup):
-        oracle_sample(inp, n_tok)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle_sample(inp, n_tok)
-    dt = (time.perf_counter() - t0) / args.steps
-    v = n_tok / dt
-    sample = (f"sequence 0 of the workload truncated to {n_tok} tokens, all {CFG.H} heads: float64 scan of K and V "
-              f"+ dense {n_tok}x{n_tok} M_test softmax attention")
+    H = CFG.H
+    for k in range(args.warmup):
+        oracle_sample(inp, heads=[k % H])
+    t0, c0 = time.perf_counter(), time.process_time()
+    for k in range(args.steps):
+        oracle_sample(inp, heads=[k % H])
+    wall, cpu = time.perf_counter() - t0, time.process_time() - c0
+    dt = wall / args.steps
+    v = (CFG.n / H) / dt
+    sample = (f"sequence 0 of the workload at its full length ({CFG.n} tokens), one of its {H} heads per step "
+              f"(heads in turn): float64 scans of K and V over that head's {CFG.dh} channels + the dense "
+              f"{CFG.n}x{CFG.n} M_test softmax attention of that head; a step counts {CFG.n}/{H} tokens")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_block(CFG, {"sample_tokens": n_tok}),
-        "cpu_baseline": {"value": v, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": sample},
+        "config": config_block(CFG),
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": effective_threads(cpu, wall),
+                         "cores_available": cpu_cores(), "kind": "oracle", "sample": sample},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
 
+def effective_threads(cpu_s, wall_s):
+    """Average number of host threads busy over a timed region (process CPU time over wall time)."""
+    return max(1, int(round(cpu_s / wall_s))) if wall_s > 0 else 1
+
+
 def cpu_baseline():
     inp = W.make_layer(CFG)
-    n_tok = 2048
-    oracle_sample(inp, 128)
-    t0 = time.perf_counter()
-    oracle_sample(inp, n_tok)
-    dt = time.perf_counter() - t0
-    return {"value": n_tok / dt, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-            "sample": f"sequence 0 truncated to {n_tok} tokens, all {CFG.H} heads, one pass "
-                      f"(float64 scan of K and V + dense M_test attention), {dt:.1f} s"}
+    t0, c0 = time.perf_counter(), time.process_time()
+    oracle_sample(inp)
+    dt, cpu = time.perf_counter() - t0, time.process_time() - c0
+    return {"value": CFG.n / dt, "unit": UNIT, "cores": effective_threads(cpu, dt),
+            "cores_available": cpu_cores(), "kind": "oracle",
+            "sample": f"sequence 0 of the workload at its full length ({CFG.n} tokens), all {CFG.H} heads, one "
+                      f"pass (float64 scans of K and V + dense {CFG.n}x{CFG.n} M_test attention), {dt:.1f} s; "
+                      f"tokens/s of one sequence (the batch's {CFG.B} sequences take {CFG.B}x as long)"}
 
 
 # ------------------------------------------------------------------ decode row
+def decode_cache_from_prefill(cfg, dec, g, dev):
+    """The decode workload's cache as the library leaves it after a prefill: a synthetic prefill of
+    ctx tokens per sequence (keys, values and scan inputs ~ N(0, 1), drawn on the device from a seeded
+    generator) handed into a cache of the workload's capacity by attamba_cache_from_prefill.
+    Returns the cache's arrays by name."""
+    from ssm_compressed_chunked_b200 import attamba as A
+    gen = torch.Generator(device=dev).manual_seed(cfg.seed)
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    B, n0, H, dh, N, L = cfg.B, cfg.ctx, cfg.H, cfg.dh, cfg.N, cfg.L
+    D = H * dh
+    cap = dec["cap"]
+    rnd = lambda *shape: torch.randn(*shape, generator=gen, device=dev, dtype=bf)  # noqa: E731
+    K, V = rnd(B, n0, H, dh), rnd(B, n0, H, dh)
+    x, dtk, dtv = rnd(B * n0, D), rnd(B * n0, D), rnd(B * n0, D)
+    bc = [rnd(B * n0, N) for _ in range(4)]
+    arrs = {"state": torch.empty(2, B, N, D, dtype=f32, device=dev),
+            "Kb": torch.empty(B, H, cap, dh, dtype=bf, device=dev), "Vb": torch.empty(B, H, cap, dh, dtype=bf, device=dev),
+            "bpos": torch.zeros(B, cap, dtype=i32, device=dev),
+            "Kr": torch.empty(B, H, L, dh, dtype=bf, device=dev), "Vr": torch.empty(B, H, L, dh, dtype=bf, device=dev),
+            "nb": torch.zeros(B, dtype=i32, device=dev), "pos": torch.zeros(B, dtype=i32, device=dev)}
+    cache = A.Cache(*(arrs[k] for k in ("state", "Kb", "Vb", "bpos", "Kr", "Vr", "nb", "pos")), cfg.P, cfg.offset)
+    status = torch.zeros(1, dtype=i32, device=dev)
+    A.cache_from_prefill(cache, K, V, x, dtk, dtv, g["bias_k"], g["bias_v"], g["A_k"], g["A_v"], *bc, n0, status)
+    torch.cuda.synchronize()
+    assert status.item() == 0, f"device status {status.item()}"
+    del K, V, x, dtk, dtv, bc
+    return arrs
+
+
 def decode_bench(dev, reps=3):
-    """128 decode steps of the decode workload (B=32, 16384 compressed tokens of context, P=8, L=64):
-    tokens/s and the HBM fraction of the whole step (cached K/V read + SSM state read/write)."""
+    """128 decode steps of the decode workload (B=32, 16384 compressed tokens of context, P=8, L=64)
+    on the cache a prefill of the context leaves: tokens/s and the HBM fraction of the whole step
+    (cached K/V read + SSM state read/write)."""
     from ssm_compressed_chunked_b200 import attamba as A
     cfg = W.DECODE_CONFIG
     dec = W.make_decode(cfg)
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in dec.items()}
-    names = ("state", "Kb", "Vb", "bpos", "Kr", "Vr", "nbuf", "pos")
-    work = {k: g[k].clone() for k in names}
-    cache = A.Cache(work["state"], work["Kb"], work["Vb"], work["bpos"], work["Kr"], work["Vr"], work["nbuf"],
-                    work["pos"], cfg.P, cfg.offset)
+    names = ("state", "Kb", "Vb", "bpos", "Kr", "Vr", "nb", "pos")
+    pristine = decode_cache_from_prefill(cfg, dec, g, dev)
+    torch.cuda.empty_cache()
+    work = {k: pristine[k].clone() for k in names}
+    cache = A.Cache(*(work[k] for k in names), cfg.P, cfg.offset)
     ws_buf = torch.empty(A.decode_workspace_size(cache), dtype=torch.uint8, device=dev)
     o = torch.empty(cfg.B, cfg.H, cfg.dh, dtype=torch.bfloat16, device=dev)
 
@@ -260,7 +310,7 @@ def decode_bench(dev, reps=3):
     times = []
     for rep in range(reps + 1):
         for k in names:
-            work[k].copy_(g[k])
+            work[k].copy_(pristine[k])
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         e0.record()
@@ -436,7 +486,7 @@ def run_ours(args, ws, rank, local):
     cfg = rank_config(CFG, ws, rank)
     inp = W.make_layer(cfg)
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
-    nch = layer.n_chunks_of(cfg, inp["cu"])
+    nch = layer.n_chunks_of(cfg)
     pf = layer.Prefill(cfg.B, cfg.n, cfg.D, cfg.H, cfg.dh, cfg.N, nch, torch.bfloat16, dev)
     mode = layer.mode_code(cfg.mode)
     stream = torch.cuda.current_stream(dev)
@@ -639,6 +689,18 @@ def run_ours(args, ws, rank, local):
     print(json.dumps(out), flush=True)
 
 
+def relaunch_ranks(n):
+    """Run this script as n ranks on this node (torch.distributed.run, rendezvous on 127.0.0.1 at a
+    free port); returns the launcher's exit status."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -652,6 +714,13 @@ def main():
     ap.add_argument("--min-warmup-ms", type=float, default=500.0,
                     help="keep warming up at least this long so clocks have ramped (0 under a profiler)")
     args = ap.parse_args()
+    if args.gpus < 1:
+        raise SystemExit("--gpus must be at least 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # one process per GPU: run this same command under torch.distributed.run with N ranks
+        sys.exit(relaunch_ranks(args.gpus))
+    if int(os.environ.get("WORLD_SIZE", "1")) != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={os.environ.get('WORLD_SIZE')}: launch one rank per GPU")
     if args.impl == "reference":
         # the CPU oracle needs no process group: rank 0 times it, other ranks exit without work
         run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))

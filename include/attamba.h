@@ -276,7 +276,9 @@ attamba_status_t attamba_decode_step(attamba_dtype_t dtype, const attamba_cache_
  *   (attamba_decode_workspace_size(cache) > 4 MiB) is rejected with
  *   ATTAMBA_ERR_UNSUPPORTED before any launch; attamba_last_error() says so.
  *   The first call on a device looks up the array's device address (no
- *   allocation); make that first call before capturing a stream.
+ *   allocation), and so does the first call after the device's context was
+ *   destroyed and created again (cudaDeviceReset); make that first call
+ *   before capturing a stream.
  *   All calls on a device share the array and it keeps the last call's
  *   contents (nothing in it needs to start at zero).  Calls whose kernels can
  *   overlap on the GPU (unordered streams) race on it; order them on one stream. */

@@ -142,14 +142,17 @@ def uniform_chunk_count(n, P, offset):
 class Index:
     """Device arrays of the compact key index (see attamba_index_t)."""
 
-    def __init__(self, n_chunks, B, n, device="cuda"):
-        i32 = dict(dtype=torch.int32, device=device)
+    def __init__(self, n_chunks, B, n, device="cuda", alloc=None):
+        """``alloc(shape, dtype)`` returns each array (default: uninitialised device memory)."""
+        if alloc is None:
+            alloc = lambda shape, dt: torch.empty(shape, dtype=dt, device=device)  # noqa: E731
+        i32 = torch.int32
         self.n_chunks, self.B, self.n = int(n_chunks), int(B), int(n)
-        self.cu = torch.empty(n_chunks + 1, **i32)
-        self.bpos = torch.empty(n_chunks, **i32)
-        self.bptr = torch.empty(B + 1, **i32)
-        self.ls = torch.empty(B * n, **i32)
-        self.nbb = torch.empty(B * n, **i32)
+        self.cu = alloc((n_chunks + 1,), i32)
+        self.bpos = alloc((n_chunks,), i32)
+        self.bptr = alloc((B + 1,), i32)
+        self.ls = alloc((B * n,), i32)
+        self.nbb = alloc((B * n,), i32)
 
     def c_struct(self):
         return IndexT(self.cu.data_ptr(), self.bpos.data_ptr(), self.bptr.data_ptr(), self.ls.data_ptr(),

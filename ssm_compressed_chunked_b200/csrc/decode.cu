@@ -197,10 +197,14 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) decode_attn_kernel(D
   }
   __syncthreads();
   const int nbb = bars->nbb;
-  const int nkeys = nbb + (t + 1 - lo);
+  const int nkeys = nbb + (t + 1 - lo);   // >= 1: the window holds t itself
+  // Splits are dealt from the end of the key list: split s covers
+  // [nkeys - (splits - s) per, nkeys - (splits - 1 - s) per) cut at 0, so the last split always
+  // holds key nkeys - 1 (position t, the ring slot its own SSM step wrote above) and any split
+  // left without keys is a leading one.  No CTA reads a slot another CTA writes in this launch.
   const int per = (nkeys + a.splits - 1) / a.splits;
-  const int kb = split * per;
-  const int ke = min(nkeys, kb + per);
+  const int ke = max(0, nkeys - (a.splits - 1 - split) * per);
+  const int kb = max(0, ke - per);
   const int nst = ke > kb ? (ke - kb + kStageKeys - 1) / kStageKeys : 0;
   const size_t bh = (size_t)b * c.H + h;
   volatile int* abort_flag = &bars->abort;
@@ -417,23 +421,61 @@ int32_t decode_splits(const attamba_cache_t& c) {
 size_t decode_noalloc_scratch_bytes() { return kNoAllocScratchFloats * sizeof(float); }
 
 // Device address of g_decode_scratch on the current device.  The name is a host
-// stand-in, not a device pointer, so the address is asked of the runtime once
-// per device (with that device current) and cached.
+// stand-in, not a device pointer, so the address is asked of the runtime (with
+// the device current) and cached.  The address belongs to the copy of this
+// library's device code loaded into the device's current context; a context
+// torn down and created again (cudaDeviceReset) loads it again, perhaps
+// elsewhere, so the cache is keyed on the context's process-unique id as well
+// as the device.  Where the driver cannot report that id, the address is asked
+// for on every call (a lookup, no allocation).
+namespace {
+bool current_context_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_current = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    return cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault, &q) == cudaSuccess &&
+                   q == cudaDriverEntryPointSuccess
+               ? reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p)
+               : nullptr;
+  }();
+  static PFN_cuCtxGetId_v12000 get_id = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    return cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+                   q == cudaDriverEntryPointSuccess
+               ? reinterpret_cast<PFN_cuCtxGetId_v12000>(p)
+               : nullptr;
+  }();
+  CUcontext ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+}  // namespace
+
 cudaError_t decode_noalloc_scratch(float** out) {
+  struct Entry {
+    unsigned long long ctx_id;
+    float* ptr;
+  };
   static std::mutex mu;
-  static float* cached[128] = {};
+  static Entry cached[128] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
-  if (cached[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess) return e;
-    cached[dev] = static_cast<float*>(p);
+  unsigned long long id = 0;
+  bool have_id = current_context_id(&id);
+  if (have_id && cached[dev].ptr != nullptr && cached[dev].ctx_id == id) {
+    *out = cached[dev].ptr;
+    return cudaSuccess;
   }
-  *out = cached[dev];
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_decode_scratch);   // makes the device's primary context current
+  if (e != cudaSuccess) return e;
+  if (!have_id) have_id = current_context_id(&id);
+  cached[dev] = have_id ? Entry{id, static_cast<float*>(p)} : Entry{0, nullptr};
+  *out = static_cast<float*>(p);
   return cudaSuccess;
 }
 

@@ -12,18 +12,25 @@ from . import attamba as A
 
 
 class Prefill:
-    def __init__(self, B, n, D, H, dh, N, n_chunks, dtype, device="cuda"):
+    """Device buffers of one prefill and the three calls over them.
+
+    ``alloc(shape, dtype)`` returns each output buffer (default: uninitialised
+    device memory); a caller can hand in its own, e.g. pre-filled memory."""
+
+    def __init__(self, B, n, D, H, dh, N, n_chunks, dtype, device="cuda", alloc=None):
         self.B, self.n, self.D, self.H, self.dh, self.N = B, n, D, H, dh, N
         self.n_chunks = n_chunks
         self.dtype = dtype
         T = B * n
-        self.index = A.Index(n_chunks, B, n, device)
-        self.K = torch.empty(T, D, dtype=dtype, device=device)
-        self.V = torch.empty(T, D, dtype=dtype, device=device)
-        self.Kc = torch.empty(n_chunks, D, dtype=dtype, device=device)
-        self.Vc = torch.empty(n_chunks, D, dtype=dtype, device=device)
-        self.O = torch.empty(T, H, dh, dtype=dtype, device=device)
-        self.lse = torch.empty(B, H, n, dtype=torch.float32, device=device)
+        if alloc is None:
+            alloc = lambda shape, dt: torch.empty(shape, dtype=dt, device=device)  # noqa: E731
+        self.index = A.Index(n_chunks, B, n, device, alloc=alloc)
+        self.K = alloc((T, D), dtype)
+        self.V = alloc((T, D), dtype)
+        self.Kc = alloc((n_chunks, D), dtype)
+        self.Vc = alloc((n_chunks, D), dtype)
+        self.O = alloc((T, H, dh), dtype)
+        self.lse = alloc((B, H, n), torch.float32)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
 
     def index_step(self, cu_in, P, offset, L, mode, stream=None):
@@ -46,7 +53,7 @@ class Prefill:
         return self.O
 
 
-def n_chunks_of(cfg, cu):
+def n_chunks_of(cfg, cu=None):
     """Chunk count of a workload: uniform from the library's count, variable from its cu array."""
     if cfg.varlen is None:
         return cfg.B * A.uniform_chunk_count(cfg.n, cfg.P, cfg.offset)

@@ -1,11 +1,14 @@
 """Seeded synthetic workloads for the Attamba layer hot path.
 
-This module only draws inputs.  It holds none of the layer's arithmetic: it
-draws the layer input and random-init weights with the distributions below,
-forms the precondition projections (q = x W_Q, dt = x W_dt, B = x W_B,
-C = x W_C, a plain fp32 matmul that lies outside the hot path), and rounds the
-results to the working dtype.  Both the CUDA path and the CPU oracle read the
-same rounded tensors.
+This module only draws inputs.  It holds none of the layer's arithmetic, and
+none of its chunking rules: it draws the layer input and random-init weights
+with the distributions below, forms the precondition projections (q = x W_Q,
+dt = x W_dt, B = x W_B, C = x W_C, a plain fp32 matmul that lies outside the
+hot path), rounds the results to the working dtype, and, for variable chunks,
+draws the chunk lengths.  Where the chunks start, which positions end one and
+what the decode cache holds are left to the caller (the tests take them from
+the oracle; the library computes them itself).  Both the CUDA path and the CPU
+oracle read the same rounded tensors.
 
 Distributions (all draws from one seeded CPU ``torch.Generator`` in this order:
 x, W_Q, W_dtK, W_dtV, W_BK, W_CK, W_BV, W_CV, W_O, A_K, A_V, dt_bias_K,
@@ -14,7 +17,8 @@ dt_bias_V, chunk lengths):
   A = -exp(U(log 1, log 16))  per (channel, state);
   dt_bias = delta0 + log(-expm1(-delta0)) with delta0 = exp(U(log 1e-3, log 1e-1)),
   the inverse of softplus, so that softplus(dt_bias) lies in [1e-3, 1e-1];
-  variable chunk lengths ~ U{lo..hi} per sequence, the running sum cut at n.
+  variable chunk lengths ~ U{lo..hi} per sequence, drawn until their sum
+  reaches n (the last one overshoots; the chunking rule cuts it at n).
 There is no dataset: the pages' quality runs (WikiText-2, dclm) are not
 reproduced; these tensors only have their shapes and value ranges.
 """
@@ -22,7 +26,6 @@ reproduced; these tensors only have their shapes and value ranges.
 from dataclasses import dataclass, replace
 import math
 
-import numpy as np
 import torch
 
 
@@ -81,33 +84,21 @@ def shrink(cfg, **kw):
     return replace(cfg, **kw)
 
 
-def _uniform_starts(n, P, offset):
-    o = offset % P
-    s = sorted({0} | {p for p in range(o, n, P) if p > 0})
-    return s
-
-
-def chunk_starts(cfg, gen):
-    """Per-sequence chunk starts (sequence-relative) for ``cfg``."""
+def draw_chunk_lengths(cfg, gen):
+    """Variable chunk lengths of each sequence, U{lo..hi}, drawn until their sum reaches n;
+    None for uniform chunks (nothing is drawn)."""
     if cfg.varlen is None:
-        return [_uniform_starts(cfg.n, cfg.P, cfg.offset) for _ in range(cfg.B)]
+        return None
     lo, hi = cfg.varlen
     out = []
     for _ in range(cfg.B):
-        starts, pos = [], 0
-        while pos < cfg.n:
-            starts.append(pos)
-            pos += int(torch.randint(lo, hi + 1, (1,), generator=gen).item())
-        out.append(starts)
+        lengths, total = [], 0
+        while total < cfg.n:
+            ln = int(torch.randint(lo, hi + 1, (1,), generator=gen).item())
+            lengths.append(ln)
+            total += ln
+        out.append(lengths)
     return out
-
-
-def cu_from_starts(starts, n):
-    cu = []
-    for b, st in enumerate(starts):
-        cu.extend(b * n + s for s in st)
-    cu.append(len(starts) * n)
-    return np.asarray(cu, dtype=np.int32)
 
 
 def _dt_bias(D, gen):
@@ -134,7 +125,8 @@ def make_layer(cfg):
 
     Returns a dict with  x, dt_k, dt_v [B, n, D];  q [B, n, H, dh];
     B_k, C_k, B_v, C_v [B, n, N];  A_k, A_v [D, N] f32;  bias_k, bias_v [D] f32;
-    starts (list per sequence);  cu int32 [n_chunks + 1];  scale = 1/sqrt(dh).
+    lengths (variable chunks: the drawn chunk lengths per sequence; else None);
+    scale = 1/sqrt(dh).
     """
     gen = torch.Generator().manual_seed(cfg.seed)
     Bsz, n, D, H, dh, N = cfg.B, cfg.n, cfg.D, cfg.H, cfg.dh, cfg.N
@@ -142,7 +134,7 @@ def make_layer(cfg):
     W = draw_weights(D, H, dh, N, gen)
     A_k, A_v = _A(D, N, gen), _A(D, N, gen)
     bias_k, bias_v = _dt_bias(D, gen), _dt_bias(D, gen)
-    starts = chunk_starts(cfg, gen)
+    lengths = draw_chunk_lengths(cfg, gen)
     dt = torch_dtype(cfg.dtype)
     xf = x.reshape(Bsz * n, D)
     proj = {k: (xf @ W[k]) for k in ("Q", "dtK", "dtV", "BK", "CK", "BV", "CV")}
@@ -156,7 +148,7 @@ def make_layer(cfg):
         B_v=r(proj["BV"], Bsz, n, N), C_v=r(proj["CV"], Bsz, n, N),
         A_k=A_k.contiguous(), A_v=A_v.contiguous(),
         bias_k=bias_k.contiguous(), bias_v=bias_v.contiguous(),
-        starts=starts, cu=cu_from_starts(starts, n),
+        lengths=lengths,
         scale=1.0 / math.sqrt(dh),
     )
 
@@ -167,12 +159,18 @@ def decode_capacity(cfg):
 
 
 def make_decode(cfg):
-    """Synthetic cache of ``cfg.ctx`` compressed tokens plus ``cfg.steps`` step inputs (CPU).
+    """Random contents for a decode cache of ``cfg.ctx`` compressed tokens plus ``cfg.steps``
+    step inputs (CPU).
 
-    Cache contents: boundary keys/values at the uniform chunk ends below ctx
-    ~ N(0, 1); the L most recent positions ~ N(0, 1), except that a boundary
-    position inside that window holds the same key/value as its boundary slot;
-    SSM states ~ N(0, 1).  Step inputs x_t ~ N(0, 1) projected like the prefill.
+    Drawn here: candidate boundary keys/values for every one of the cache's boundary slots,
+    keys/values for the L ring slots, and the SSM states, all ~ N(0, 1); step inputs
+    x_t ~ N(0, 1) projected like the prefill.  Which slots hold a boundary (the positions
+    below ctx that end a chunk) and which ring slots repeat a boundary is the chunking rule,
+    left to the caller.
+
+    Returns Kb, Vb [B, H, cap, dh];  Kr, Vr [B, H, L, dh];  state [2, B, N, D] f32;
+    x, dt_k, dt_v [steps, B, D];  q [steps, B, H, dh];  B_k .. C_v [steps, B, N];
+    A_k, A_v, bias_k, bias_v as in make_layer;  cap;  scale.
     """
     gen = torch.Generator().manual_seed(cfg.seed)
     Bsz, D, H, dh, N, L = cfg.B, cfg.D, cfg.H, cfg.dh, cfg.N, cfg.L
@@ -181,33 +179,20 @@ def make_decode(cfg):
     W = draw_weights(D, H, dh, N, gen)
     A_k, A_v = _A(D, N, gen), _A(D, N, gen)
     bias_k, bias_v = _dt_bias(D, gen), _dt_bias(D, gen)
-    o = cfg.offset % cfg.P
-    bpos = [p for p in range(cfg.ctx) if p + 1 >= o and (p + 1 - o) % cfg.P == 0]
-    nb = len(bpos)
     cap = decode_capacity(cfg)
-    Kb = torch.zeros(Bsz, H, cap, dh, dtype=dt)
-    Vb = torch.zeros(Bsz, H, cap, dh, dtype=dt)
-    Kb[:, :, :nb] = torch.randn(Bsz, H, nb, dh, generator=gen).to(dt)
-    Vb[:, :, :nb] = torch.randn(Bsz, H, nb, dh, generator=gen).to(dt)
+    Kb = torch.randn(Bsz, H, cap, dh, generator=gen).to(dt)
+    Vb = torch.randn(Bsz, H, cap, dh, generator=gen).to(dt)
     Kr = torch.randn(Bsz, H, L, dh, generator=gen).to(dt)
     Vr = torch.randn(Bsz, H, L, dh, generator=gen).to(dt)
-    for k, p in enumerate(bpos):
-        if p >= cfg.ctx - L:
-            Kr[:, :, p % L] = Kb[:, :, k]
-            Vr[:, :, p % L] = Vb[:, :, k]
     state = torch.randn(2, Bsz, N, D, generator=gen)
-    bpos_t = torch.zeros(Bsz, cap, dtype=torch.int32)
-    bpos_t[:, :nb] = torch.tensor(bpos, dtype=torch.int32)
     xf = xs.reshape(cfg.steps * Bsz, D)
     proj = {k: (xf @ W[k]) for k in ("Q", "dtK", "dtV", "BK", "CK", "BV", "CV")}
     r = lambda t, *shape: t.reshape(*shape).to(dt).contiguous()
     S = cfg.steps
     return dict(
-        cfg=cfg, cap=cap, nb=nb,
+        cfg=cfg, cap=cap,
         state=state.contiguous(),                # [2, B, N, D] f32 (state-major per channel)
-        Kb=Kb, Vb=Vb, bpos=bpos_t, Kr=Kr, Vr=Vr,
-        pos=torch.full((Bsz,), cfg.ctx, dtype=torch.int32),
-        nbuf=torch.full((Bsz,), nb, dtype=torch.int32),
+        Kb=Kb, Vb=Vb, Kr=Kr, Vr=Vr,
         x=r(xs, S, Bsz, D),
         q=r(proj["Q"], S, Bsz, H, dh),
         dt_k=r(proj["dtK"], S, Bsz, D), dt_v=r(proj["dtV"], S, Bsz, D),

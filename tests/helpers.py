@@ -1,10 +1,25 @@
-"""Shared test plumbing: run the CUDA path on a workload and run the oracle on the same inputs."""
+"""Shared test plumbing: run the CUDA path on a workload and run the oracle on the same inputs.
+
+The chunk layout of a workload (where its chunks start, which positions end
+one, what a decode cache holds) always comes from the oracle's own rules
+(``oracle.chunks``, ``oracle.decode``); the workload generator only draws
+random values and chunk lengths.
+
+Every buffer a kernel writes in these tests is poisoned first and followed by a
+guard region (``Guarded``): outputs start as a NaN canary (0xA5A5A5A5 for
+int32), so a value a kernel leaves unwritten fails the comparison instead of
+passing on memory an earlier test left behind, and a write past the end of an
+array shows up as a changed guard.  These stand in for a memory checker.
+"""
+
+import math
 
 import numpy as np
 import torch
 
 from oracle import attention as OA
 from oracle import chunks as OC
+from oracle import decode as OD
 from oracle import mask as OM
 from oracle import ssm as OS
 from ssm_compressed_chunked_b200 import layer
@@ -76,25 +91,92 @@ def attn_rounding_bound(q, K, V, O, key_lists, scale):
     return out
 
 
+# ------------------------------------------------------------------ chunk layout from the oracle
+def chunk_starts(inp):
+    """Sequence-relative chunk starts of each sequence of a workload, by the oracle's rules:
+    uniform chunks (size P, cyclic offset) or the drawn variable lengths cut at n."""
+    cfg = inp["cfg"]
+    if cfg.varlen is None:
+        return [OC.uniform_starts(cfg.n, cfg.P, cfg.offset) for _ in range(cfg.B)]
+    return [OC.varlen_starts(lengths, cfg.n) for lengths in inp["lengths"]]
+
+
+def cu_of(inp):
+    """cu_seqlens-style chunk starts over the B sequences laid end to end (int32)."""
+    return OC.flatten_batch(chunk_starts(inp), inp["cfg"].n).astype(np.int32)
+
+
+# ------------------------------------------------------------------ poisoned, guarded outputs
+GUARD = 256   # guard elements after every array
+_CANARY = {torch.bfloat16: (torch.int16, 0x7FA5),            # a NaN
+           torch.float32: (torch.int32, 0x7FA5A5A5),          # a NaN
+           torch.int32: (torch.int32, -0x5A5A5A5B)}           # 0xA5A5A5A5, never a valid index
+
+
+def poison_(t):
+    """Fill t with its dtype's canary (NaN for floats, 0xA5A5A5A5 for int32) in place."""
+    iv, pat = _CANARY[t.dtype]
+    t.view(iv).fill_(pat)
+    return t
+
+
+class Guarded:
+    """Allocator of poisoned output buffers, each followed by GUARD canary elements."""
+
+    def __init__(self, device="cuda"):
+        self.device = device
+        self.bufs = []
+
+    def __call__(self, shape, dtype):
+        numel = math.prod(shape)
+        buf = poison_(torch.empty(numel + GUARD, dtype=dtype, device=self.device))
+        self.bufs.append((buf, numel))
+        return buf[:numel].view(shape)
+
+    def check(self):
+        """Every guard region still holds the canary (no write past the end of an array)."""
+        for buf, numel in self.bufs:
+            iv, pat = _CANARY[buf.dtype]
+            g = buf[numel:].view(iv)
+            assert bool((g == pat).all()), f"guard after a {tuple(buf.shape)} {buf.dtype} array was written"
+
+
+def assert_written(t, what):
+    """No element of t still holds the canary: the kernel wrote all of it."""
+    if t.dtype == torch.int32:
+        assert bool((t != _CANARY[torch.int32][1]).all()), f"{what}: entries left unwritten"
+    else:
+        assert not bool(torch.isnan(t).any()), f"{what}: NaN (unwritten) entries"
+
+
 def to_gpu(inp):
     out = {}
     for k, v in inp.items():
         out[k] = v.cuda() if isinstance(v, torch.Tensor) else v
-    out["cu_t"] = torch.from_numpy(inp["cu"]).cuda()
+    out["cu"] = cu_of(inp)
+    out["cu_t"] = torch.from_numpy(out["cu"]).cuda()
     return out
 
 
 def run_prefill(inp, cfg):
-    """CUDA path on a workload dict (CPU tensors); returns the Prefill object (device buffers)."""
+    """CUDA path on a workload dict (CPU tensors) into poisoned, guarded buffers; checks the guards
+    and that every output element was written, and returns the Prefill object (device buffers)."""
     g = to_gpu(inp)
-    nch = layer.n_chunks_of(cfg, inp["cu"])
-    pf = layer.Prefill(cfg.B, cfg.n, cfg.D, cfg.H, cfg.dh, cfg.N, nch, W.torch_dtype(cfg.dtype))
+    nch = layer.n_chunks_of(cfg, g["cu"])
+    guard = Guarded()
+    pf = layer.Prefill(cfg.B, cfg.n, cfg.D, cfg.H, cfg.dh, cfg.N, nch, W.torch_dtype(cfg.dtype), alloc=guard)
     cu_in = g["cu_t"] if cfg.varlen is not None else None
     P = cfg.P if cfg.varlen is None else 1
     pf.forward(g["x"], g["q"], g["dt_k"], g["dt_v"], g["bias_k"], g["bias_v"], g["A_k"], g["A_v"],
                g["B_k"], g["C_k"], g["B_v"], g["C_v"], cu_in, P, cfg.offset, cfg.L, layer.mode_code(cfg.mode),
                inp["scale"])
     torch.cuda.synchronize()
+    pf.guard = guard
+    guard.check()
+    for name in ("K", "V", "Kc", "Vc", "O", "lse"):
+        assert_written(getattr(pf, name), name)
+    for name in ("cu", "bpos", "bptr", "ls", "nbb"):
+        assert_written(getattr(pf.index, name), "index." + name)
     return pf
 
 
@@ -104,7 +186,7 @@ def oracle_scan_seq(inp, b, t0=None, t1=None):
     n = cfg.n
     t0 = 0 if t0 is None else t0
     t1 = n if t1 is None else t1
-    starts = np.asarray(inp["starts"][b])
+    starts = np.asarray(chunk_starts(inp)[b])
     is_start = OC.is_start_mask(starts, n)[t0:t1]
     assert is_start[0]
     sl = slice(t0, t1)
@@ -126,3 +208,119 @@ def oracle_attention_seq(q, K, V, starts, n, L, mode, scale, rows=None):
     if rows is None:
         return OA.masked_attention(q, K, V, OM.dense_mask(n, starts, L, mode), scale)
     return OA.attention_rows(q, K, V, rows, key_lists(n, starts, L, mode, rows), scale)
+
+
+# ------------------------------------------------------------------ decode caches
+def decode_cache_contents(dec):
+    """The synthetic decode cache of ``W.make_decode`` laid out by the oracle's chunk-end rule:
+    boundaries at the positions below ctx that end a chunk (their rows from the drawn candidates,
+    the rows past them poisoned with NaN so a read past nb shows), ring slots of window positions
+    that are boundaries holding the boundary's key/value, pos = ctx.  CPU tensors."""
+    cfg = dec["cfg"]
+    bpos = [p for p in range(cfg.ctx) if OD.is_chunk_end(p, cfg.P, cfg.offset)]
+    nb, cap = len(bpos), dec["cap"]
+    assert nb <= cap
+    Kb, Vb = dec["Kb"].clone(), dec["Vb"].clone()
+    Kb[:, :, nb:] = float("nan")
+    Vb[:, :, nb:] = float("nan")
+    Kr, Vr = dec["Kr"].clone(), dec["Vr"].clone()
+    for k, p in enumerate(bpos):
+        if p >= cfg.ctx - cfg.L:
+            Kr[:, :, p % cfg.L] = Kb[:, :, k]
+            Vr[:, :, p % cfg.L] = Vb[:, :, k]
+    bp = torch.full((cfg.B, cap), -1, dtype=torch.int32)
+    bp[:, :nb] = torch.tensor(bpos, dtype=torch.int32)
+    return dict(state=dec["state"].clone(), Kb=Kb, Vb=Vb, bpos=bp, Kr=Kr, Vr=Vr,
+                nb=torch.full((cfg.B,), nb, dtype=torch.int32),
+                pos=torch.full((cfg.B,), cfg.ctx, dtype=torch.int32))
+
+
+_CACHE_ARRAYS = ("state", "Kb", "Vb", "bpos", "Kr", "Vr", "nb", "pos")
+
+
+def gpu_cache(contents, P, offset, guard=None):
+    """A device cache (attamba.Cache) holding copies of ``contents``; each array inside a guarded
+    buffer when ``guard`` (a Guarded) is given."""
+    from ssm_compressed_chunked_b200 import attamba as A
+    arrs = {}
+    for k in _CACHE_ARRAYS:
+        src = contents[k]
+        if guard is None:
+            arrs[k] = src.cuda().clone()
+        else:
+            t = guard(tuple(src.shape), src.dtype)
+            t.copy_(src)
+            arrs[k] = t
+    return A.Cache(*(arrs[k] for k in _CACHE_ARRAYS), P, offset)
+
+
+def empty_cache_contents(B, H, dh, N, L, cap):
+    """An empty decode cache (no boundaries, position 0); unwritten rows poisoned with NaN / -1."""
+    D = H * dh
+    bf = torch.bfloat16
+    return dict(state=torch.full((2, B, N, D), float("nan")),
+                Kb=torch.full((B, H, cap, dh), float("nan"), dtype=bf),
+                Vb=torch.full((B, H, cap, dh), float("nan"), dtype=bf),
+                bpos=torch.full((B, cap), -1, dtype=torch.int32),
+                Kr=torch.full((B, H, L, dh), float("nan"), dtype=bf),
+                Vr=torch.full((B, H, L, dh), float("nan"), dtype=bf),
+                nb=torch.zeros(B, dtype=torch.int32), pos=torch.zeros(B, dtype=torch.int32))
+
+
+def oracle_cache(contents, cfg, rows):
+    """A cache's contents (CPU tensors) in the oracle's format, for the batch rows ``rows``."""
+    c = OD.DecodeCache(len(rows), cfg.H, cfg.dh, cfg.N, cfg.P, cfg.offset, cfg.L)
+    c.state = np.transpose(f64(contents["state"][:, rows]), (0, 1, 3, 2)).copy()
+    for r, b in enumerate(rows):
+        nb = int(contents["nb"][b])
+        t = int(contents["pos"][b])
+        c.bpos[r] = contents["bpos"][b, :nb].tolist()
+        Kb = f64(contents["Kb"][b, :, :nb])
+        Vb = f64(contents["Vb"][b, :, :nb])
+        c.Kb[r] = [Kb[:, k] for k in range(nb)]
+        c.Vb[r] = [Vb[:, k] for k in range(nb)]
+        for p in range(max(0, t - cfg.L), t):
+            c.ring[r][p] = (f64(contents["Kr"][b, :, p % cfg.L]), f64(contents["Vr"][b, :, p % cfg.L]))
+        c.pos[r] = t
+    return c
+
+
+def oracle_step(oc, dec_or_inp, s, rows, scale, col=None):
+    """One oracle decode step for the batch rows ``rows`` on step s's inputs.
+
+    ``dec_or_inp`` holds per-step arrays [steps, B, ...] (col None) or prefill arrays
+    [B, n, ...] read at position ``col``."""
+    def sel(name):
+        t = dec_or_inp[name]
+        return f64(t[s][rows]) if col is None else f64(t[rows, col])
+    return oc.step(sel("q"), sel("x"), np.stack([sel("dt_k"), sel("dt_v")]),
+                   np.stack([f64(dec_or_inp["bias_k"]), f64(dec_or_inp["bias_v"])]),
+                   np.stack([f64(dec_or_inp["A_k"]), f64(dec_or_inp["A_v"])]),
+                   np.stack([sel("B_k"), sel("B_v")]), np.stack([sel("C_k"), sel("C_v")]), scale)
+
+
+def decode_rounding_bound(oc, r, q, o_ref, ctx, scale):
+    """First-order effect on a decode output of keys the GPU stored in bf16 while the oracle keeps
+    them in float64: the keys and values at positions >= ctx (those the GPU computed; rows of a
+    synthetic bf16 cache are the same on both sides).  Same rule as the prefill attention's: a
+    change dv moves o by at most max |dv|, a change dk moves a score by at most scale sum |q| |dk|
+    and o by at most max |v - o| times that.  Returns [H, dh] for batch row r of the oracle cache."""
+    t = oc.pos[r] - 1
+    lo = max(0, t - oc.L + 1)
+    ks, vs = [], []
+    for p, kk, vv in zip(oc.bpos[r], oc.Kb[r], oc.Vb[r]):
+        if ctx <= p < lo:
+            ks.append(kk)
+            vs.append(vv)
+    for p in range(max(lo, ctx), t + 1):
+        kk, vv = oc.ring[r][p]
+        ks.append(kk)
+        vs.append(vv)
+    if not ks:
+        return np.zeros_like(o_ref)
+    k = np.stack(ks)                                               # [j, H, dh]
+    v = np.stack(vs)
+    ds = scale * BF16_HALF_ULP * np.einsum("hd,jhd->jh", np.abs(q), np.abs(k)).max(axis=0)    # [H]
+    dv = BF16_HALF_ULP * np.abs(v).max(axis=0)                                                 # [H, dh]
+    spread = np.abs(v - o_ref[None]).max(axis=0)
+    return dv + spread * ds[:, None]

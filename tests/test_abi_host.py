@@ -7,8 +7,8 @@ import re
 
 import pytest
 
+from oracle import chunks as OC
 from ssm_compressed_chunked_b200 import attamba as A
-from ssm_compressed_chunked_b200 import workloads as W
 
 HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "attamba.h")
 
@@ -36,8 +36,8 @@ def test_version_and_status_strings():
 
 @pytest.mark.parametrize("n,P,o", [(10, 4, 0), (10, 4, 3), (256, 4, 0), (2048, 4, 3), (4096, 8, 0), (1, 4, 2),
                                    (7, 1, 0), (9, 8, 7), (16, 16, 0)])
-def test_uniform_chunk_count_matches_workload_starts(n, P, o):
-    assert A.uniform_chunk_count(n, P, o) == len(W._uniform_starts(n, P, o))
+def test_uniform_chunk_count_matches_oracle_starts(n, P, o):
+    assert A.uniform_chunk_count(n, P, o) == len(OC.uniform_starts(n, P, o))
 
 
 def test_invalid_arguments_are_rejected_on_the_host():

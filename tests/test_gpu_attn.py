@@ -10,8 +10,8 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import (assert_close, attn_rounding_bound, f64, key_lists, oracle_attention_seq, oracle_scan_seq,
-                     run_prefill)
+from helpers import (assert_close, assert_written, attn_rounding_bound, chunk_starts, f64, key_lists,
+                     oracle_attention_seq, oracle_scan_seq, poison_, run_prefill)
 from ssm_compressed_chunked_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -45,8 +45,9 @@ def test_attention_small(cfg):
     lse = pf.lse.cpu().numpy()
     K = pf.K.view(cfg.B, n, H, dh)
     V = pf.V.view(cfg.B, n, H, dh)
+    starts = chunk_starts(inp)
     for b in range(cfg.B):
-        st = np.asarray(inp["starts"][b])
+        st = np.asarray(starts[b])
         q = f64(inp["q"][b])
         # stage-isolated: oracle attention over the GPU's own K/V
         ro, rl = oracle_attention_seq(q, f64(K[b]), f64(V[b]), st, n, cfg.L, cfg.mode, inp["scale"])
@@ -78,8 +79,9 @@ def test_attention_wide_score_range(qscale):
     lse = pf.lse.cpu().numpy()
     K = pf.K.view(cfg.B, n, H, dh)
     V = pf.V.view(cfg.B, n, H, dh)
+    starts = chunk_starts(inp)
     for b in range(cfg.B):
-        st = np.asarray(inp["starts"][b])
+        st = np.asarray(starts[b])
         ro, rl = oracle_attention_seq(f64(inp["q"][b]), f64(K[b]), f64(V[b]), st, n, cfg.L, cfg.mode, inp["scale"])
         assert_close(cfg.dtype, f64(O[b]), ro, f"O (q x {qscale}) b={b}")
         fin = np.isfinite(rl)
@@ -99,7 +101,7 @@ def test_attention_full_size_sampled_rows(cfg):
     V = pf.V.view(cfg.B, n, H, dh)
     rng = np.random.default_rng(7)
     b = cfg.B - 1
-    st = np.asarray(inp["starts"][b])
+    st = np.asarray(chunk_starts(inp)[b])
     rows = sorted({0, 1, 127, 128, n - 129, n - 1} | set(rng.integers(0, n, size=26).tolist()))
     q = f64(inp["q"][b])
     ro, _ = oracle_attention_seq(q, f64(K[b]), f64(V[b]), st, n, cfg.L, cfg.mode, inp["scale"], rows)
@@ -119,8 +121,11 @@ def test_value_one_gives_output_one():
     pf = run_prefill(inp, cfg)
     pf.V.fill_(1.0)
     pf.Vc.fill_(1.0)
+    poison_(pf.O)
     pf.attn_step(inp["q"].cuda(), inp["scale"])
     torch.cuda.synchronize()
+    pf.guard.check()
+    assert_written(pf.O, "O")
     np.testing.assert_allclose(f64(pf.O), 1.0, atol=1e-2)
 
 
@@ -138,4 +143,5 @@ def test_attention_without_lse(cfg):
                      pf.index, inp["scale"], O2, None, pf.status)
     torch.cuda.synchronize()
     assert pf.status.item() == 0
+    assert_written(O2, "O without lse")
     assert torch.equal(O2, pf.O)

@@ -7,6 +7,7 @@ import numpy as np
 import pytest
 import torch
 
+from helpers import cu_of
 from ssm_compressed_chunked_b200 import attamba as A, layer, workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -24,12 +25,13 @@ def test_bounded_wait_gives_up_and_reports():
     # the context is still usable: a prefill chunk index right after matches the uniform layout
     cfg = W.shrink(W.BF16_TEST_P8_L64, B=2, n=300, D=128, H=2)
     inp = W.make_layer(cfg)
-    nch = layer.n_chunks_of(cfg, inp["cu"])
+    cu = cu_of(inp)
+    nch = layer.n_chunks_of(cfg, cu)
     pf = layer.Prefill(cfg.B, cfg.n, cfg.D, cfg.H, cfg.dh, cfg.N, nch, torch.bfloat16)
     pf.index_step(None, cfg.P, cfg.offset, cfg.L, layer.mode_code(cfg.mode))
     torch.cuda.synchronize()
     assert pf.status.item() == 0
-    np.testing.assert_array_equal(pf.index.cu[: nch + 1].cpu().numpy(), np.asarray(inp["cu"], dtype=np.int32))
+    np.testing.assert_array_equal(pf.index.cu[: nch + 1].cpu().numpy(), cu)
 
 
 def test_status_bits_accumulate_across_calls():

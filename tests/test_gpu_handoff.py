@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import BF16_ATOL, f64, run_prefill
+from helpers import BF16_ATOL, Guarded, assert_written, empty_cache_contents, f64, gpu_cache, run_prefill
 from oracle import chunks as OC
 from oracle import decode as OD
 from oracle import ssm as OS
@@ -18,18 +18,6 @@ from ssm_compressed_chunked_b200 import attamba as A
 from ssm_compressed_chunked_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
-
-
-def _empty_cache(B, H, dh, N, P, offset, L, cap):
-    dev = "cuda"
-    return A.Cache(torch.full((2, B, N, H * dh), float("nan"), device=dev),
-                   torch.zeros(B, H, cap, dh, dtype=torch.bfloat16, device=dev),
-                   torch.zeros(B, H, cap, dh, dtype=torch.bfloat16, device=dev),
-                   torch.full((B, cap), -1, dtype=torch.int32, device=dev),
-                   torch.zeros(B, H, L, dh, dtype=torch.bfloat16, device=dev),
-                   torch.zeros(B, H, L, dh, dtype=torch.bfloat16, device=dev),
-                   torch.zeros(B, dtype=torch.int32, device=dev), torch.zeros(B, dtype=torch.int32, device=dev),
-                   P, offset)
 
 
 @pytest.mark.parametrize("P,offset,L,n0,N", [(8, 3, 16, 300, 16), (4, 0, 8, 256, 16), (8, 0, 64, 40, 16),
@@ -47,12 +35,15 @@ def test_cache_from_prefill_matches_oracle_and_continues_the_prefill(P, offset, 
     V0 = pf.V.view(B, n, H, dh)[:, :n0].contiguous()
     flat = lambda t: head(t).view(B * n0, -1)
     cap = n // P + 2
-    cache = _empty_cache(B, H, dh, N, P, offset, L, cap)
+    guard = Guarded()
+    cache = gpu_cache(empty_cache_contents(B, H, dh, N, L, cap), P, offset, guard)   # NaN until written
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     A.cache_from_prefill(cache, K0, V0, flat(g["x"]), flat(g["dt_k"]), flat(g["dt_v"]), g["bias_k"], g["bias_v"],
                          g["A_k"], g["A_v"], flat(g["B_k"]), flat(g["C_k"]), flat(g["B_v"]), flat(g["C_v"]), n0, status)
     torch.cuda.synchronize()
     assert status.item() == 0
+    guard.check()
+    assert_written(cache.state, "state")
 
     # bookkeeping and copied rows against the oracle's rule
     ends = [p for p in range(n0) if OD.is_chunk_end(p, P, offset)]
@@ -79,11 +70,12 @@ def test_cache_from_prefill_matches_oracle_and_continues_the_prefill(P, offset, 
     ws = torch.empty(A.decode_workspace_size(cache), dtype=torch.uint8, device="cuda")
     O_pre = pf.O.view(B, n, H, dh)
     for t in range(n0, n):
-        o = torch.empty(B, H, dh, dtype=torch.bfloat16, device="cuda")
+        o = guard((B, H, dh), torch.bfloat16)
         c = lambda name: g[name][:, t].contiguous()
         A.decode_step(cache, c("q"), c("x"), c("dt_k"), c("dt_v"), g["bias_k"], g["bias_v"], g["A_k"], g["A_v"],
                       c("B_k"), c("C_k"), c("B_v"), c("C_v"), inp["scale"], o, ws, status)
         err = (o.float() - O_pre[:, t].float()).abs().max().item()
         assert err <= BF16_ATOL, (t, err)
     torch.cuda.synchronize()
+    guard.check()
     assert status.item() == 0

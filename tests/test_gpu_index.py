@@ -4,6 +4,7 @@ import numpy as np
 import pytest
 import torch
 
+from helpers import Guarded, assert_written, chunk_starts
 from oracle import chunks as OC
 from oracle import mask as OM
 from ssm_compressed_chunked_b200 import attamba as A
@@ -15,9 +16,10 @@ pytestmark = pytest.mark.gpu
 
 def _gpu_index(starts_per_seq, n, L, mode, uniform=None):
     B = len(starts_per_seq)
-    cu = W.cu_from_starts([list(s) for s in starts_per_seq], n)
+    cu = OC.flatten_batch(starts_per_seq, n).astype(np.int32)
     nch = len(cu) - 1
-    idx = A.Index(nch, B, n)
+    guard = Guarded()
+    idx = A.Index(nch, B, n, alloc=guard)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     if uniform is None:
         A.chunk_index(torch.from_numpy(cu).cuda(), nch, B, n, 1, 0, L, mode, idx, status)
@@ -26,6 +28,9 @@ def _gpu_index(starts_per_seq, n, L, mode, uniform=None):
         A.chunk_index(None, nch, B, n, P, o, L, mode, idx, status)
     torch.cuda.synchronize()
     assert status.item() == 0
+    guard.check()
+    for name in ("cu", "bpos", "bptr", "ls", "nbb"):
+        assert_written(getattr(idx, name), name)
     return cu, idx
 
 
@@ -72,9 +77,7 @@ def test_random_sweep():
 
 @pytest.mark.parametrize("cfg", W.LAYER_CONFIGS, ids=lambda c: c.name)
 def test_configs(cfg):
-    gen = torch.Generator().manual_seed(cfg.seed)
-    starts = W.chunk_starts(cfg, gen) if cfg.varlen is not None else \
-        [W._uniform_starts(cfg.n, cfg.P, cfg.offset)] * cfg.B
+    starts = chunk_starts(W.make_layer(cfg))
     uniform = None if cfg.varlen is not None else (cfg.P, cfg.offset)
     cu, idx = _gpu_index(starts, cfg.n, cfg.L, layer.mode_code(cfg.mode), uniform)
     _check(starts, cfg.n, cfg.L, cfg.mode, idx, cu, dense=cfg.n <= 2048)

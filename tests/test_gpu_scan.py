@@ -4,7 +4,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import assert_close, f64, oracle_scan_seq, run_prefill
+from helpers import Guarded, assert_close, assert_written, chunk_starts, f64, oracle_scan_seq, run_prefill
 from oracle import chunks as OC
 from ssm_compressed_chunked_b200 import workloads as W
 
@@ -35,7 +35,7 @@ def test_scan_small(cfg):
         assert_close(cfg.dtype, f64(K[b]), rk, f"K b={b}")
         assert_close(cfg.dtype, f64(V[b]), rv, f"V b={b}")
     # chunk-end rows are the same values as the full outputs at the chunk ends (bit-exact copy)
-    ends = np.array([b * cfg.n + e for b, st in enumerate(inp["starts"]) for e in OC.boundary_positions(st, cfg.n)])
+    ends = np.array([b * cfg.n + e for b, st in enumerate(chunk_starts(inp)) for e in OC.boundary_positions(st, cfg.n)])
     assert torch.equal(pf.Kc, pf.K[torch.from_numpy(ends).cuda()])
     assert torch.equal(pf.Vc, pf.V[torch.from_numpy(ends).cuda()])
     assert pf.status.item() == 0
@@ -50,7 +50,7 @@ def test_scan_full_size_sampled_chunks(cfg):
     V = pf.V.view(cfg.B, cfg.n, cfg.D)
     rng = np.random.default_rng(cfg.seed)
     for b in (0, cfg.B - 1):
-        st = list(inp["starts"][b]) + [cfg.n]
+        st = list(chunk_starts(inp)[b]) + [cfg.n]
         picks = {0, len(st) - 2} | set(rng.integers(0, len(st) - 1, size=4).tolist())
         for c in sorted(picks):
             t0, t1 = st[c], st[c + 1]
@@ -78,22 +78,26 @@ def test_scan_kept_projection_inputs(cfg):
     x32 = inp["x"].float().reshape(-1, cfg.D)
     u = [(x32 @ w).to(dt) for w in proj]                     # the caller's projections, rounded like q
     T = cfg.B * cfg.n
-    K = torch.empty(T, cfg.D, dtype=dt, device="cuda")
-    V = torch.empty_like(K)
+    guard = Guarded()
+    K = guard((T, cfg.D), dt)
+    V = guard((T, cfg.D), dt)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     flat = lambda t: t.reshape(T, -1)
     args = (flat(g["dt_k"]), flat(g["dt_v"]), g["bias_k"], g["bias_v"], g["A_k"], g["A_v"], flat(g["B_k"]),
             flat(g["C_k"]), flat(g["B_v"]), flat(g["C_v"]), pf.index.cu, pf.n_chunks)
     A.kv_ssm_scan_u(u[0].cuda(), u[1].cuda(), *args, K, V, status=status)
     # shared input through the new entry point equals the original one exactly
-    K2 = torch.empty_like(K)
-    V2 = torch.empty_like(K)
+    K2 = guard((T, cfg.D), dt)
+    V2 = guard((T, cfg.D), dt)
     A.kv_ssm_scan_u(flat(g["x"]), flat(g["x"]), *args, K2, V2, status=status)
     torch.cuda.synchronize()
     assert status.item() == 0
+    guard.check()
+    for name, t in (("K", K), ("V", V), ("K2", K2), ("V2", V2)):
+        assert_written(t, name)
     assert torch.equal(K2, pf.K) and torch.equal(V2, pf.V)
     for b in range(cfg.B):
-        is_start = OC.is_start_mask(np.asarray(inp["starts"][b]), cfg.n)
+        is_start = OC.is_start_mask(np.asarray(chunk_starts(inp)[b]), cfg.n)
         sl = slice(b * cfg.n, (b + 1) * cfg.n)
         for s, name, out in ((0, "k", K), (1, "v", V)):
             ref, _ = OS.selective_scan(f64(u[s][sl]), f64(inp["dt_" + name][b]), f64(inp["bias_" + name]),

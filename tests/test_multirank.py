@@ -66,3 +66,21 @@ def test_reference_arm_prints_the_contract_line(capsys):
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_gpus_flag_relaunches_one_rank_per_gpu(monkeypatch):
+    """bench.py --gpus N started without a launcher runs itself as N ranks; under a launcher the
+    world size must match N."""
+    import sys
+    import bench
+    calls = []
+    monkeypatch.setattr(bench, "relaunch_ranks", lambda n: calls.append(n) or 0)
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--gpus", "2", "--steps", "3"])
+    with pytest.raises(SystemExit) as e:
+        bench.main()
+    assert e.value.code == 0 and calls == [2]
+    monkeypatch.setenv("WORLD_SIZE", "4")
+    with pytest.raises(SystemExit) as e:
+        bench.main()
+    assert "WORLD_SIZE=4" in str(e.value.code)
