@@ -120,6 +120,19 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(win), "source": "NVML, 0.5 ms period"}
 
 
+class nvtx:
+    """An NVTX range (torch's binding) around a block, so a timeline tool shows each C-ABI call by name."""
+
+    def __init__(self, name):
+        self.name = name
+
+    def __enter__(self):
+        torch.cuda.nvtx.range_push(self.name)
+
+    def __exit__(self, *exc):
+        torch.cuda.nvtx.range_pop()
+
+
 def source_sha(files):
     h = hashlib.sha256()
     for f in files:
@@ -303,9 +316,10 @@ def decode_bench(dev, reps=3):
 
     def steps():
         for st in range(cfg.steps):
-            A.decode_step(cache, g["q"][st], g["x"][st], g["dt_k"][st], g["dt_v"][st], g["bias_k"], g["bias_v"],
-                          g["A_k"], g["A_v"], g["B_k"][st], g["C_k"][st], g["B_v"][st], g["C_v"][st], dec["scale"],
-                          o, ws_buf)
+            with nvtx("attamba_decode_step"):
+                A.decode_step(cache, g["q"][st], g["x"][st], g["dt_k"][st], g["dt_v"][st], g["bias_k"],
+                              g["bias_v"], g["A_k"], g["A_v"], g["B_k"][st], g["C_k"][st], g["B_v"][st], g["C_v"][st],
+                              dec["scale"], o, ws_buf)
 
     times = []
     for rep in range(reps + 1):
@@ -496,18 +510,21 @@ def run_ours(args, ws, rank, local):
         """One step: chunk_index, kv_ssm_scan, chunk_attn_fwd on the inputs `src` (default: the
         resident set).  Two events bracket the step; four also split it per call (an event between two
         calls keeps the second call's launch from overlapping the first call's tail, so the split sums
-        to a little more than the step)."""
+        to a little more than the step).  Each C-ABI call sits in an NVTX range of its name."""
         src = g if src is None else src
         if events:
             events[0].record(stream)
-        pf.index_step(None, cfg.P, cfg.offset, cfg.L, mode)
+        with nvtx("attamba_chunk_index"):
+            pf.index_step(None, cfg.P, cfg.offset, cfg.L, mode)
         if events and len(events) == 4:
             events[1].record(stream)
-        pf.scan_step(src["x"], src["dt_k"], src["dt_v"], g["bias_k"], g["bias_v"], g["A_k"], g["A_v"], src["B_k"],
-                     src["C_k"], src["B_v"], src["C_v"])
+        with nvtx("attamba_kv_ssm_scan"):
+            pf.scan_step(src["x"], src["dt_k"], src["dt_v"], g["bias_k"], g["bias_v"], g["A_k"], g["A_v"],
+                         src["B_k"], src["C_k"], src["B_v"], src["C_v"])
         if events and len(events) == 4:
             events[2].record(stream)
-        pf.attn_step(src["q"], inp["scale"])
+        with nvtx("attamba_chunk_attn_fwd"):
+            pf.attn_step(src["q"], inp["scale"])
         if events:
             events[-1].record(stream)
 

@@ -68,6 +68,10 @@ typedef enum { ATTAMBA_MASK_TRAIN = 0, ATTAMBA_MASK_TEST = 1 } attamba_mask_t;
 #define ATTAMBA_DEV_BAD_CHUNKS 0x1 /* cu not increasing, not 0..T, or a chunk crosses a sequence start */
 #define ATTAMBA_DEV_CACHE_FULL 0x2 /* decode: boundary list at capacity, the new boundary was dropped */
 #define ATTAMBA_DEV_TIMEOUT 0x4    /* a pipeline wait gave up; outputs of that tile are not written */
+#define ATTAMBA_DEV_BOUNDS 0x8     /* checked builds only (libattamba_checked.so, compiled with
+                                      ATTAMBA_CHECKED): an index fell outside the array it addresses;
+                                      the access was skipped (a TMA load, which reads the fill value
+                                      out of range, is reported and still made) */
 
 /* Compact per-query key index built by attamba_chunk_index [pith, carries]:
  * query i (sequence-relative position) of sequence b reads

@@ -14,12 +14,15 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libattamba.so")
+# ATTAMBA_LIBRARY=checked selects the bounds-checked build (libattamba_checked.so): the same kernels
+# with every index tested against its array, a failure reported as DEV_BOUNDS in the status word
+LIB_PATH = os.path.join(_HERE, "libattamba_checked.so" if os.environ.get("ATTAMBA_LIBRARY") == "checked"
+                        else "libattamba.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA = 0, 1, 2, 3
 F32, BF16 = 0, 1
 MASK_TRAIN, MASK_TEST = 0, 1
-DEV_BAD_CHUNKS, DEV_CACHE_FULL, DEV_TIMEOUT = 0x1, 0x2, 0x4
+DEV_BAD_CHUNKS, DEV_CACHE_FULL, DEV_TIMEOUT, DEV_BOUNDS = 0x1, 0x2, 0x4, 0x8
 
 # every symbol include/attamba.h declares
 EXPORTS = ("attamba_version", "attamba_status_string", "attamba_last_error",

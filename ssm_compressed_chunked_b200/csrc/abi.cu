@@ -20,7 +20,13 @@ constexpr int64_t kMaxTokens = (int64_t)1 << 31;
 
 extern "C" {
 
-const char* attamba_version(void) { return "attamba-b200 0.1 (sm_100a)"; }
+const char* attamba_version(void) {
+#if defined(ATTAMBA_CHECKED)
+  return "attamba-b200 0.1 (sm_100a) checked";
+#else
+  return "attamba-b200 0.1 (sm_100a)";
+#endif
+}
 
 const char* attamba_status_string(attamba_status_t s) {
   switch (s) {

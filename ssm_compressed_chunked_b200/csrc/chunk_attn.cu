@@ -158,6 +158,11 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a, int item, int n_q
   const int band_len = band_empty ? 0 : max(0, it.q_last - it.ls_first + 1);
   it.NT = it.nbt + (band_len + kBN - 1) / kBN;
   it.chunk0 = a.bptr[it.b];
+  // the item's chunk-end tiles read the sequence's own chunk ends, its band starts inside the sequence
+  if (!in_bounds(a.nbb[tok0 + it.q_last] <= a.bptr[it.b + 1] - it.chunk0 && it.ls_first >= 0 &&
+                     it.ls_first <= it.q0 + 1 && it.q_last < a.n,
+                 a.status))
+    it.NT = 0;
   return it;
 }
 
@@ -419,6 +424,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       if (row_ok) {
         my_ls = a.ls[tok0 + i];
         my_nbb = a.nbb[tok0 + i];
+        // the row's keys lie inside the item's tiles (the chunk-end tiles cover nbb(q_last) >= nbb(i),
+        // the band starts at ls(first query) <= ls(i))
+        if (!in_bounds(my_nbb <= it.nbt * kBN && my_ls >= it.ls_first, a.status)) {
+          my_nbb = 0;
+          my_ls = i + 1;
+        }
       }
       if (it.NT == 0) {  // every row of the item has an empty key set
         if (row_ok) {

@@ -37,6 +37,19 @@ __device__ __forceinline__ void raise_status(int32_t* st, int bits) {
   if (st) atomicOr(st, bits);
 }
 
+// Checked builds (compiled with ATTAMBA_CHECKED) test index computations against
+// the bounds of the arrays they address: a failed test ORs ATTAMBA_DEV_BOUNDS into
+// the status word and the caller skips the access.  In normal builds the test is
+// the constant true and the condition is never evaluated at run time.
+#if defined(ATTAMBA_CHECKED)
+__device__ __forceinline__ bool in_bounds(bool ok, int32_t* st) {
+  if (!ok) raise_status(st, ATTAMBA_DEV_BOUNDS);
+  return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool in_bounds(bool, int32_t*) { return true; }
+#endif
+
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

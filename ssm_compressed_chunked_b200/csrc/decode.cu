@@ -113,6 +113,7 @@ __device__ __forceinline__ void ssm_step(const DecodeArgs& a, int s, int b, int 
   const int D = c.H * c.dh;
   const int o = ((c.offset % c.P) + c.P) % c.P;
   const int t = a.c.pos[b];
+  if (!in_bounds(t >= 0, a.status)) return;   // a position below 0 has no ring slot
   const bool start = chunk_starts_at(t, c.P, o);
   const bool end = chunk_ends_at(t, c.P, o);
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(a.x);
@@ -205,7 +206,9 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) decode_attn_kernel(D
   const int per = (nkeys + a.splits - 1) / a.splits;
   const int ke = max(0, nkeys - (a.splits - 1 - split) * per);
   const int kb = max(0, ke - per);
-  const int nst = ke > kb ? (ke - kb + kStageKeys - 1) / kStageKeys : 0;
+  // the boundary rows read lie below the stored count and the capacity, the window starts at 0 or later
+  const bool rows_ok = in_bounds(t >= 0 && nbb <= min(max(c.nb[b], 0), cap) && kb >= 0 && ke <= nkeys, a.status);
+  const int nst = (rows_ok && ke > kb) ? (ke - kb + kStageKeys - 1) / kStageKeys : 0;
   const size_t bh = (size_t)b * c.H + h;
   volatile int* abort_flag = &bars->abort;
 

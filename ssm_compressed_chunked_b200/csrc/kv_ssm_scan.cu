@@ -276,6 +276,8 @@ __global__ void __launch_bounds__(kScanThreads, MINB) kv_ssm_scan_kernel(ScanArg
   __syncthreads();
   const int t_begin = sCu[0];
   const int t_end = sCu[c_end - c_begin];
+  // every thread reads the same offsets, so a failed check returns the whole block before its barriers
+  if (!in_bounds(t_begin >= 0 && t_begin < t_end && (int64_t)t_end <= p.T && c_end <= p.n_chunks, p.status)) return;
   int ci = 0;                 // chunk of the current token, relative to c_begin
   int next_start = sCu[1];
 
@@ -314,7 +316,8 @@ __global__ void __launch_bounds__(kScanThreads, MINB) kv_ssm_scan_kernel(ScanArg
     float y[CPT];
     scan_token<T, CPT, NS, POLY_PAIRS>(st, bc, dl, dx, reset, poly_ok, y);
     V::store(out + t * D, y);
-    if (outc != nullptr && t + 1 == next_start) V::store(outc + (c_begin + ci) * D + d0, y);
+    if (outc != nullptr && t + 1 == next_start && in_bounds(c_begin + ci < p.n_chunks, p.status))
+      V::store(outc + (c_begin + ci) * D + d0, y);
   };
 
   for (int tb = t_begin; tb < t_end; tb += kStageTokens) {

@@ -27,6 +27,16 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(lib, name), name
 
 
+def test_checked_library_exports_every_declared_symbol():
+    """The bounds-checked build (ATTAMBA_CHECKED) exports the same C ABI and says so in its version."""
+    path = os.path.join(os.path.dirname(A.LIB_PATH), "libattamba_checked.so")
+    lib = ctypes.CDLL(path)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    lib.attamba_version.restype = ctypes.c_char_p
+    assert lib.attamba_version().endswith(b"checked")
+
+
 def test_version_and_status_strings():
     assert "sm_100a" in A.version()
     lib = A.load()
