@@ -298,12 +298,13 @@ def decode_cache_from_prefill(cfg, dec, g, dev):
     return arrs
 
 
-def decode_bench(dev, reps=3):
+def decode_bench(dev, reps=3, batch=None):
     """128 decode steps of the decode workload (B=32, 16384 compressed tokens of context, P=8, L=64)
     on the cache a prefill of the context leaves: tokens/s and the HBM fraction of the whole step
-    (cached K/V read + SSM state read/write)."""
+    (cached K/V read + SSM state read/write).  ``batch`` runs the same workload with another batch
+    size (a smaller case for profiler captures)."""
     from ssm_compressed_chunked_b200 import attamba as A
-    cfg = W.DECODE_CONFIG
+    cfg = W.DECODE_CONFIG if batch is None else W.shrink(W.DECODE_CONFIG, B=batch)
     dec = W.make_decode(cfg)
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in dec.items()}
     names = ("state", "Kb", "Vb", "bpos", "Kr", "Vr", "nb", "pos")
@@ -698,7 +699,8 @@ def run_ours(args, ws, rank, local):
         "clocks": clocks,
     }
     if ws == 1 and not args.no_decode:
-        out["decode"] = decode_bench(dev)
+        out["decode"] = decode_bench(dev, batch=args.decode_batch)
+        torch.cuda.empty_cache()   # the decode caches go back to the driver before the next rows
     if ws == 1 and not args.no_next_rows:
         out["next_rows"] = next_rows_bench(cfg, g, inp, pf, nch, dev, flush, scan_exps)
     if ws == 1 and not args.no_cpu_baseline:
@@ -730,6 +732,10 @@ def main():
                     help="skip timing the rows built after the hot path (kept projections, N = 32, handoff)")
     ap.add_argument("--min-warmup-ms", type=float, default=500.0,
                     help="keep warming up at least this long so clocks have ramped (0 under a profiler)")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="time only the decode row and print it (a profiler capture of the decode kernels)")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="batch size of the decode row (default: the workload's 32)")
     args = ap.parse_args()
     if args.gpus < 1:
         raise SystemExit("--gpus must be at least 1")
@@ -738,6 +744,10 @@ def main():
         sys.exit(relaunch_ranks(args.gpus))
     if int(os.environ.get("WORLD_SIZE", "1")) != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={os.environ.get('WORLD_SIZE')}: launch one rank per GPU")
+    if args.decode_only:
+        torch.cuda.set_device(0)
+        print(json.dumps({"decode": decode_bench(torch.device("cuda", 0), batch=args.decode_batch)}), flush=True)
+        return
     if args.impl == "reference":
         # the CPU oracle needs no process group: rank 0 times it, other ranks exit without work
         run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))

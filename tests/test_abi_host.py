@@ -92,6 +92,37 @@ def test_invalid_arguments_are_rejected_on_the_host():
     assert lib.attamba_selftest_wait_timeout(1000000001, fake, None) == A.ERR_INVALID_ARG
 
 
+def test_scan_refuses_sizes_past_its_offset_limit():
+    """The scan addresses [T, D] with 32-bit element offsets: T * D = 2^31 is refused on the host,
+    before any launch (the pointers are never dereferenced)."""
+    lib = A.load()
+    fake = 1 << 20
+    D = 1024
+    T = (1 << 31) // D
+    st = lib.attamba_kv_ssm_scan(A.BF16, *([fake] * 12), 1, T, D, 16, fake, fake, None, None, None, None)
+    assert st == A.ERR_UNSUPPORTED
+
+
+def test_empty_inputs_are_refused():
+    """No sequence, no token or no chunk: every entry point rejects the call before any launch."""
+    lib = A.load()
+    fake = 1 << 20
+    idx = A.IndexT(fake, fake, fake, fake, fake, 1, 1, 0)
+    assert lib.attamba_chunk_index(None, 1, 1, 0, 4, 0, 0, 0, ctypes.byref(idx), None, None) == A.ERR_INVALID_ARG
+    idx0 = A.IndexT(fake, fake, fake, fake, fake, 0, 0, 16)
+    assert lib.attamba_chunk_index(None, 0, 0, 16, 4, 0, 0, 0, ctypes.byref(idx0), None, None) == A.ERR_INVALID_ARG
+    assert lib.attamba_kv_ssm_scan(A.BF16, *([fake] * 12), 1, 0, 64, 16, fake, fake, None, None, None,
+                                   None) == A.ERR_INVALID_ARG
+    assert lib.attamba_kv_ssm_scan(A.BF16, *([fake] * 12), 0, 16, 64, 16, fake, fake, None, None, None,
+                                   None) == A.ERR_INVALID_ARG
+    assert lib.attamba_chunk_attn_fwd(A.BF16, fake, fake, fake, fake, fake, ctypes.byref(idx), 2, 64,
+                                      ctypes.c_float(0.1), fake, None, None, None) == A.ERR_INVALID_ARG
+    c = A.CacheT(*([fake] * 8), 0, 1, 64, 16, 8, 0, 4, 16)
+    assert lib.attamba_decode_step(A.BF16, ctypes.byref(c), *([fake] * 12), ctypes.c_float(0.1), fake, fake,
+                                   1 << 20, None, None) == A.ERR_INVALID_ARG
+    assert lib.attamba_proj_gemm(A.BF16, fake, fake, 0, 64, 64, None, 0, None, None) == A.ERR_INVALID_ARG
+
+
 def test_cpu_tensors_are_refused():
     import torch
     with pytest.raises(A.AttambaError):
