@@ -79,7 +79,6 @@ attamba_status_t scan_entry(attamba_dtype_t dtype, const void* u_k, const void* 
   if (N != 16 && N != 32) return ATTAMBA_ERR_UNSUPPORTED;
   if (T < 1 || T >= kMaxTokens || D < 8 || D % 8 != 0 || n_chunks < 1 || n_chunks > T)
     return ATTAMBA_ERR_INVALID_ARG;
-  if (T * D >= kMaxTokens) return ATTAMBA_ERR_UNSUPPORTED;  // element offsets are 32-bit
   const void* req[] = {u_k, u_v, dt_k, dt_v, bias_k, bias_v, A_k, A_v, B_k, C_k, B_v, C_v, cu, K, V};
   for (const void* p : req)
     if (!p || !aligned16(p)) return ATTAMBA_ERR_INVALID_ARG;

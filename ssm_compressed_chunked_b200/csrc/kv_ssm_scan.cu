@@ -35,6 +35,8 @@
 // it, like an FMA-pipe softplus or skipping the decay at chunk starts behind a
 // branch, was slower: the unit is busy, but the FMA pipe and the instruction
 // schedule (one basic block per token pair) are close behind.
+#include <type_traits>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -230,8 +232,11 @@ __device__ __forceinline__ void scan_unit(const ScanGrid& gr, int32_t n_chunks, 
   c_end = min(c_begin + gr.size[ph], ph < 2 ? gr.start[ph + 1] : n_chunks);
 }
 
-template <typename T, int CPT, int NS, int POLY_PAIRS, int MINB, bool SPLIT_X>
+// WIDE: element offsets into the [T, D] and [T, N] arrays in 64 bits (T * D or T * N >= 2^31);
+// otherwise in 32 bits, which the token loop issues fewer instructions for.
+template <typename T, int CPT, int NS, int POLY_PAIRS, int MINB, bool SPLIT_X, bool WIDE>
 __global__ void __launch_bounds__(kScanThreads, MINB) kv_ssm_scan_kernel(ScanArgs p, ScanGrid gr) {
+  using Off = typename std::conditional<WIDE, int64_t, int32_t>::type;
   using V = Vec<T, CPT>;
   constexpr int kNS = NS;
   constexpr int kNP = NS / 2;
@@ -244,7 +249,7 @@ __global__ void __launch_bounds__(kScanThreads, MINB) kv_ssm_scan_kernel(ScanArg
   int xg, s;
   int32_t c_begin, c_end;
   scan_unit(gr, p.n_chunks, xg, s, c_begin, c_end);
-  const int D = p.D;  // T * D < 2^31 (checked by the host): 32-bit element offsets
+  const Off D = p.D;  // element offsets t * D in 32 bits unless WIDE
   const int d0 = (xg * kScanThreads + threadIdx.x) * CPT;
   const bool active = d0 < D;
   if (c_begin >= c_end) return;
@@ -325,8 +330,8 @@ __global__ void __launch_bounds__(kScanThreads, MINB) kv_ssm_scan_kernel(ScanArg
     if (tb != t_begin) __syncthreads();
     for (int e = threadIdx.x; e < nt * kNS; e += kScanThreads) {
       const int k = e / kNS, n = e - k * kNS;
-      sBC[k][n] = Elem<T>::to_f(Bm[(tb + k) * kNS + n]);
-      sBC[k][kNS + n] = Elem<T>::to_f(Cm[(tb + k) * kNS + n]);
+      sBC[k][n] = Elem<T>::to_f(Bm[(Off)(tb + k) * kNS + n]);
+      sBC[k][kNS + n] = Elem<T>::to_f(Cm[(Off)(tb + k) * kNS + n]);
     }
     __syncthreads();
     if (!active) continue;
@@ -346,7 +351,7 @@ __global__ void __launch_bounds__(kScanThreads, MINB) kv_ssm_scan_kernel(ScanArg
 
 namespace {
 // N = 16: two channels per thread; N = 32: one (the state and A of two channels would not fit)
-template <int NS, int CPT, int MINB, bool SPLIT_X>
+template <int NS, int CPT, int MINB, bool SPLIT_X, bool WIDE>
 cudaError_t launch_scan(attamba_dtype_t dtype, const ScanArgs& a, cudaStream_t s) {
   // about ATTAMBA_SCAN_TOKENS tokens of chunks per full unit; the chunks after the first
   // ATTAMBA_SCAN_F1 percent in half and quarter units
@@ -382,17 +387,26 @@ cudaError_t launch_scan(attamba_dtype_t dtype, const ScanArgs& a, cudaStream_t s
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (dtype == ATTAMBA_BF16)
-    return cudaLaunchKernelEx(&cfg, kv_ssm_scan_kernel<__nv_bfloat16, CPT, NS, NS == 16 ? ATTAMBA_SCAN_POLY_PAIRS : 0, MINB, SPLIT_X>,
-                              a, gr);
-  return cudaLaunchKernelEx(&cfg, kv_ssm_scan_kernel<float, CPT, NS, 0, MINB, SPLIT_X>, a, gr);
+    return cudaLaunchKernelEx(
+        &cfg, kv_ssm_scan_kernel<__nv_bfloat16, CPT, NS, NS == 16 ? ATTAMBA_SCAN_POLY_PAIRS : 0, MINB, SPLIT_X, WIDE>, a,
+        gr);
+  return cudaLaunchKernelEx(&cfg, kv_ssm_scan_kernel<float, CPT, NS, 0, MINB, SPLIT_X, WIDE>, a, gr);
+}
+
+template <bool WIDE>
+cudaError_t launch_scan_offsets(attamba_dtype_t dtype, const ScanArgs& a, cudaStream_t s) {
+  const bool split = a.x[0] != a.x[1];
+  if (a.N == 32)
+    return split ? launch_scan<32, 1, 3, true, WIDE>(dtype, a, s) : launch_scan<32, 1, 3, false, WIDE>(dtype, a, s);
+  return split ? launch_scan<16, ATTAMBA_SCAN_CPT, ATTAMBA_SCAN_MINB, true, WIDE>(dtype, a, s)
+               : launch_scan<16, ATTAMBA_SCAN_CPT, ATTAMBA_SCAN_MINB, false, WIDE>(dtype, a, s);
 }
 }  // namespace
 
 cudaError_t launch_kv_ssm_scan(attamba_dtype_t dtype, const ScanArgs& a, cudaStream_t s) {
-  const bool split = a.x[0] != a.x[1];
-  if (a.N == 32) return split ? launch_scan<32, 1, 3, true>(dtype, a, s) : launch_scan<32, 1, 3, false>(dtype, a, s);
-  return split ? launch_scan<16, ATTAMBA_SCAN_CPT, ATTAMBA_SCAN_MINB, true>(dtype, a, s)
-               : launch_scan<16, ATTAMBA_SCAN_CPT, ATTAMBA_SCAN_MINB, false>(dtype, a, s);
+  // 32-bit element offsets while they can address every element, 64-bit beyond
+  const bool wide = a.T * a.D >= ((int64_t)1 << 31) || a.T * a.N >= ((int64_t)1 << 31);
+  return wide ? launch_scan_offsets<true>(dtype, a, s) : launch_scan_offsets<false>(dtype, a, s);
 }
 
 }  // namespace attamba

@@ -92,17 +92,6 @@ def test_invalid_arguments_are_rejected_on_the_host():
     assert lib.attamba_selftest_wait_timeout(1000000001, fake, None) == A.ERR_INVALID_ARG
 
 
-def test_scan_refuses_sizes_past_its_offset_limit():
-    """The scan addresses [T, D] with 32-bit element offsets: T * D = 2^31 is refused on the host,
-    before any launch (the pointers are never dereferenced)."""
-    lib = A.load()
-    fake = 1 << 20
-    D = 1024
-    T = (1 << 31) // D
-    st = lib.attamba_kv_ssm_scan(A.BF16, *([fake] * 12), 1, T, D, 16, fake, fake, None, None, None, None)
-    assert st == A.ERR_UNSUPPORTED
-
-
 def test_empty_inputs_are_refused():
     """No sequence, no token or no chunk: every entry point rejects the call before any launch."""
     lib = A.load()

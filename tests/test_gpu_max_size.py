@@ -1,12 +1,13 @@
-"""The hot path at the largest size its 32-bit element offsets allow (GPU).
+"""The hot path on either side of the scan's switch to 64-bit offsets (GPU).
 
-The scan addresses [T, D] arrays with 32-bit element offsets, so the library
-refuses T * D >= 2^31 (ATTAMBA_ERR_UNSUPPORTED).  Here one sequence of
-n = 2^21 - 64 tokens at d_model 1024 (T * D = 2^31 - 65536) runs through the
-chunk index, both scans and the attention under M_test (P = 4096, L = 64, so
-each query reads up to 511 chunk ends plus 64 window keys).  The oracle checks
-sampled chunks and query rows, the last ones among them, where the offsets come
-closest to the limit.  Inputs are drawn on the device from a seeded generator
+The scan addresses the [T, D] arrays with 32-bit element offsets while
+T * D < 2^31 and with 64-bit ones beyond (a second instantiation).  Here one
+sequence of n = 2^21 - 64 tokens at d_model 1024 (T * D = 2^31 - 65536, the
+32-bit form) and one of n = 2^21 + 64 (T * D = 2^31 + 65536, the 64-bit form)
+run through the chunk index, both scans and the attention under M_test (P =
+4096, L = 64, so each query reads up to 512 chunk ends plus 64 window keys).
+The oracle checks sampled chunks and query rows, the last ones among them,
+where the offsets are largest.  Inputs are drawn on the device from a seeded generator
 (N(0, 1), like the projected workload tensors); A and the step bias follow the
 workload recipe.  Every output buffer is poisoned and guarded.
 """
@@ -26,14 +27,14 @@ from ssm_compressed_chunked_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
 
-N_TOK = (1 << 21) - 64
 D, H, DH, NS, P, L = 1024, 16, 64, 16, 4096, 64
 
 
-def test_hot_path_at_the_offset_limit():
-    B, n = 1, N_TOK
+@pytest.mark.parametrize("n", [(1 << 21) - 64, (1 << 21) + 64], ids=["32-bit offsets", "64-bit offsets"])
+def test_hot_path_at_the_offset_limit(n):
+    B = 1
     T = B * n
-    assert T * D < 2 ** 31 <= (T + 2 * P) * D
+    assert abs(T * D - 2 ** 31) == 64 * D
     bf = torch.bfloat16
     gen = torch.Generator(device="cuda").manual_seed(2024)
     rnd = lambda *shape: torch.randn(*shape, generator=gen, device="cuda", dtype=bf)  # noqa: E731
