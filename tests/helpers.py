@@ -5,11 +5,12 @@ one, what a decode cache holds) always comes from the oracle's own rules
 (``oracle.chunks``, ``oracle.decode``); the workload generator only draws
 random values and chunk lengths.
 
-Every buffer a kernel writes in these tests is poisoned first and followed by a
-guard region (``Guarded``): outputs start as a NaN canary (0xA5A5A5A5 for
+Every buffer a kernel writes in these tests is poisoned first and placed between
+two guard regions (``Guarded``): outputs start as a NaN canary (0xA5A5A5A5 for
 int32), so a value a kernel leaves unwritten fails the comparison instead of
-passing on memory an earlier test left behind, and a write past the end of an
-array shows up as a changed guard.  These stand in for a memory checker.
+passing on memory an earlier test left behind, and a write before the start or
+past the end of an array shows up as a changed guard.  These stand in for a
+memory checker.
 """
 
 import math
@@ -121,7 +122,10 @@ def poison_(t):
 
 
 class Guarded:
-    """Allocator of poisoned output buffers, each followed by GUARD canary elements."""
+    """Allocator of poisoned output buffers, each between two runs of GUARD canary elements.
+
+    The array starts GUARD elements into its buffer (512 bytes or more, so every 16-byte alignment the
+    library asks for holds)."""
 
     def __init__(self, device="cuda"):
         self.device = device
@@ -129,16 +133,18 @@ class Guarded:
 
     def __call__(self, shape, dtype):
         numel = math.prod(shape)
-        buf = poison_(torch.empty(numel + GUARD, dtype=dtype, device=self.device))
+        buf = poison_(torch.empty(numel + 2 * GUARD, dtype=dtype, device=self.device))
         self.bufs.append((buf, numel))
-        return buf[:numel].view(shape)
+        return buf[GUARD:GUARD + numel].view(shape)
 
     def check(self):
-        """Every guard region still holds the canary (no write past the end of an array)."""
+        """Both guard regions of every array still hold the canary (no write before its start or past
+        its end)."""
         for buf, numel in self.bufs:
             iv, pat = _CANARY[buf.dtype]
-            g = buf[numel:].view(iv)
-            assert bool((g == pat).all()), f"guard after a {tuple(buf.shape)} {buf.dtype} array was written"
+            for where, g in (("before", buf[:GUARD]), ("after", buf[GUARD + numel:])):
+                assert bool((g.view(iv) == pat).all()), \
+                    f"guard {where} a {numel}-element {buf.dtype} array was written"
 
 
 def assert_written(t, what):
