@@ -442,15 +442,14 @@ def next_rows_bench(cfg, g, inp, pf, nch, dev, flush, scan_exps, reps=10):
     # pinned host memory and y copied back every step (copies on streams of their own, two x buffers,
     # so step k + 1's x crosses PCIe while step k computes)
     from ssm_compressed_chunked_b200 import layer
-    mode = layer.mode_code(cfg.mode)
-    q_, dtk_, dtv_, bk_, ck_, bv_, cv_ = [o for o, _ in outs]
+    weights = {name: blk for name, blk in zip(layer.INPUT_PROJECTIONS, torch.split(W_in, widths, dim=0))}
+    weights.update(W_O=W_O, bias_k=g["bias_k"], bias_v=g["bias_v"], A_k=g["A_k"], A_v=g["A_v"])
+    lay = layer.Layer(cfg.B, cfg.n, D, H, dh, cfg.N, weights, cfg.P, cfg.offset, cfg.L, layer.mode_code(cfg.mode),
+                      inp["scale"], device=dev)
+    y = lay.y
 
     def layer_fwd(xs):
-        A.proj_gemm(xs, W_in, outs, pf.status)
-        pf.index_step(None, cfg.P, cfg.offset, cfg.L, mode)
-        pf.scan_step(xs, dtk_, dtv_, g["bias_k"], g["bias_v"], g["A_k"], g["A_v"], bk_, ck_, bv_, cv_)
-        pf.attn_step(q_.view(T, H, dh), inp["scale"])
-        A.proj_gemm(pf.O.view(T, H * dh), W_O, [(y, 0)], pf.status)
+        lay.forward(xs)
 
     ms_layer = timed(lambda: layer_fwd(flat(g["x"])))
     h_x = inp["x"].reshape(T, D).pin_memory()
@@ -489,7 +488,8 @@ def next_rows_bench(cfg, g, inp, pf, nch, dev, flush, scan_exps, reps=10):
         "us": ms_layer * 1e3, "tokens_per_s": T / (ms_layer * 1e-3),
         "e2e_tokens_per_s": T / (ms_e2e * 1e-3), "h2d_bytes_per_step": T * D * 2, "d2h_bytes_per_step": T * D * 2,
         "note": "x in, y = O W_O out; random-init projection weights of the workload's shapes"}
-    assert pf.status.item() == 0, f"device status {pf.status.item()}"
+    assert pf.status.item() == 0 and lay.status.item() == 0, \
+        f"device status {pf.status.item()}, layer {lay.status.item()}"
     return rows
 
 

@@ -1,6 +1,9 @@
-"""The prefill hot path as three C-ABI calls on preallocated device buffers.
+"""The prefill hot path as three C-ABI calls on preallocated device buffers,
+and the whole layer with its projections around it.
 
     chunk_index  ->  kv_ssm_scan (K and V, plus the chunk-end rows Kc, Vc)  ->  chunk_attn_fwd
+
+    Layer:  x  --proj_gemm-->  q, dt_K, dt_V, B_K, C_K, B_V, C_V  --hot path-->  O  --proj_gemm-->  y = O W_O
 
 Only buffer allocation happens here (torch, once); every step of the path runs
 in libattamba.so.
@@ -62,3 +65,72 @@ def n_chunks_of(cfg, cu=None):
 
 def mode_code(mode):
     return A.MASK_TRAIN if mode == "train" else A.MASK_TEST
+
+
+# the layer's input projections, in the column order of the one GEMM that computes them
+INPUT_PROJECTIONS = ("W_Q", "W_dtK", "W_dtV", "W_BK", "W_CK", "W_BV", "W_CV")
+
+
+class Layer:
+    """One Attamba layer forward, y = Attn(q, K, V) W_O, on preallocated device buffers.
+
+    pith.science review of Attamba, "Core claim": the keys and values come from
+    two SSMs over the layer input (K = SSM_K(x), V = SSM_V(x)) in place of W_K
+    and W_V, while the query and output projections stay; "Assumptions & free
+    parameters": each SSM is Mamba's selective SSM, whose step and B, C are
+    projections of its input.  So x is projected seven ways (q, dt_K, dt_V, B_K,
+    C_K, B_V, C_V) by one GEMM whose column segments land in the arrays the hot
+    path reads, the hot path gives O, and a second GEMM gives y = O W_O.
+
+    ``weights`` maps each name of INPUT_PROJECTIONS and "W_O" to a bf16 matrix in
+    [out, in] layout (W_Q [H dh, D]; W_dtK, W_dtV [D, D]; W_BK ... W_CV [N, D];
+    W_O [D, H dh]) and "bias_k", "bias_v" [D], "A_k", "A_v" [D, N] to fp32; all on
+    the layer's device.  The chunking is uniform (P, offset) unless ``forward``
+    gets chunk offsets ``cu_in``; ``mode`` is MASK_TEST or MASK_TRAIN."""
+
+    def __init__(self, B, n, D, H, dh, N, weights, P, offset, L, mode, scale, n_chunks=None, device="cuda",
+                 alloc=None):
+        bf = torch.bfloat16
+        self.B, self.n, self.D, self.H, self.dh, self.N = B, n, D, H, dh, N
+        self.P, self.offset, self.L, self.mode, self.scale = P, offset, L, mode, scale
+        T = B * n
+        shapes = {"W_Q": (H * dh, D), "W_dtK": (D, D), "W_dtV": (D, D), "W_BK": (N, D), "W_CK": (N, D),
+                  "W_BV": (N, D), "W_CV": (N, D), "W_O": (D, H * dh)}
+        for name, shape in shapes.items():
+            w = weights[name]
+            if tuple(w.shape) != shape or w.dtype != bf:
+                raise A.AttambaError(f"{name} must be bf16 {shape}, got {w.dtype} {tuple(w.shape)}")
+        self.W_in = torch.cat([weights[k] for k in INPUT_PROJECTIONS], dim=0).contiguous()
+        self.W_O = weights["W_O"].contiguous()
+        self.bias_k, self.bias_v = weights["bias_k"], weights["bias_v"]
+        self.A_k, self.A_v = weights["A_k"], weights["A_v"]
+        if alloc is None:
+            alloc = lambda shape, dt: torch.empty(shape, dtype=dt, device=device)  # noqa: E731
+        widths = [shapes[k][0] for k in INPUT_PROJECTIONS]
+        self.proj, c = [], 0
+        for w in widths:
+            self.proj.append((alloc((T, w), bf), c))
+            c += w
+        if n_chunks is None:
+            n_chunks = B * A.uniform_chunk_count(n, P, offset)
+        self.prefill = Prefill(B, n, D, H, dh, N, n_chunks, bf, device=device, alloc=alloc)
+        self.y = alloc((T, D), bf)
+        self.status = self.prefill.status
+
+    @property
+    def projections(self):
+        """The projected activations, by the names of INPUT_PROJECTIONS without the "W_"."""
+        return {k[2:]: t for k, (t, _) in zip(INPUT_PROJECTIONS, self.proj)}
+
+    def forward(self, x, cu_in=None, stream=None):
+        """x [B n, D] bf16 -> y [B n, D] bf16 (the layer's own buffer)."""
+        T, H, dh = self.B * self.n, self.H, self.dh
+        q, dt_k, dt_v, B_k, C_k, B_v, C_v = (t for t, _ in self.proj)
+        A.proj_gemm(x, self.W_in, self.proj, self.status, stream)
+        pf = self.prefill
+        pf.index_step(cu_in, self.P if cu_in is None else 1, self.offset, self.L, self.mode, stream)
+        pf.scan_step(x, dt_k, dt_v, self.bias_k, self.bias_v, self.A_k, self.A_v, B_k, C_k, B_v, C_v, stream)
+        pf.attn_step(q.view(T, H, dh), self.scale, stream)
+        A.proj_gemm(pf.O.view(T, H * dh), self.W_O, [(self.y, 0)], self.status, stream)
+        return self.y
+

@@ -77,11 +77,13 @@ def test_proj_gemm_more_tiles_than_resident_pairs():
         _check(t.cpu(), r, X, W[sum(widths[:k]):sum(widths[:k + 1])], f"segment {k}")
 
 
-def test_proj_gemm_layer_size_sampled_rows():
-    """The layer's input projections at the bench size (M = 4 x 4096 tokens, K = 1024, seven
-    segments): 96 sampled rows against the oracle's float64 product of those rows."""
-    M, K, widths = 16384, 1024, [1024, 1024, 1024, 16, 16, 16, 16]
-    gen = torch.Generator().manual_seed(12)
+@pytest.mark.parametrize("widths", [[1024, 1024, 1024, 16, 16, 16, 16], [1024]], ids=["inputs", "output"])
+def test_proj_gemm_layer_size_sampled_rows(widths):
+    """The layer's projections at the bench size (M = 4 x 4096 tokens, K = 1024): the seven input
+    segments (q, dt_K, dt_V, B_K, C_K, B_V, C_V) and the output projection O W_O.  Every element is
+    written (the outputs start as NaN); 96 sampled rows match the oracle's float64 product."""
+    M, K = 16384, 1024
+    gen = torch.Generator().manual_seed(12 + len(widths))
     Nout = sum(widths)
     X = torch.randn(M, K, generator=gen).to(torch.bfloat16)
     W = (torch.randn(Nout, K, generator=gen) / K ** 0.5).to(torch.bfloat16)
@@ -93,6 +95,8 @@ def test_proj_gemm_layer_size_sampled_rows():
     A.proj_gemm(X.cuda(), W.cuda(), outs, status)
     torch.cuda.synchronize()
     assert status.item() == 0
+    for k, (t, _) in enumerate(outs):
+        assert not torch.isnan(t).any().item(), f"segment {k} has unwritten elements"
     rows = torch.randperm(M, generator=gen)[:96].sort().values
     Xs = X[rows]
     ref = OP.split(OP.project(f64(Xs), f64(W)), widths)
