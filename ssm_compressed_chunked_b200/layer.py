@@ -86,7 +86,13 @@ class Layer:
     [out, in] layout (W_Q [H dh, D]; W_dtK, W_dtV [D, D]; W_BK ... W_CV [N, D];
     W_O [D, H dh]) and "bias_k", "bias_v" [D], "A_k", "A_v" [D, N] to fp32; all on
     the layer's device.  The chunking is uniform (P, offset) unless ``forward``
-    gets chunk offsets ``cu_in``; ``mode`` is MASK_TEST or MASK_TRAIN."""
+    gets chunk offsets ``cu_in``; ``mode`` is MASK_TEST or MASK_TRAIN.
+
+    Decoding (pith.science review, "Core claim": the inference cache holds the
+    chunk boundary states, and "If this is right": P = 8 with 64 leading tokens)
+    continues a uniform-chunk prefill one token at a time under M_test:
+    ``new_cache`` or ``cache_from_prefill`` gives the cache, ``decode_step`` maps
+    x_t to y_t."""
 
     def __init__(self, B, n, D, H, dh, N, weights, P, offset, L, mode, scale, n_chunks=None, device="cuda",
                  alloc=None):
@@ -121,6 +127,58 @@ class Layer:
     def projections(self):
         """The projected activations, by the names of INPUT_PROJECTIONS without the "W_"."""
         return {k[2:]: t for k, (t, _) in zip(INPUT_PROJECTIONS, self.proj)}
+
+    # ---------------------------------------------------------------- decode (M_test, uniform chunks)
+    def new_cache(self, cap, device="cuda"):
+        """An empty decode cache (every sequence at position 0) with room for ``cap`` chunk-end rows
+        per sequence and the layer's L most recent tokens, chunked like the layer (P, offset)."""
+        if self.L < 1:
+            raise A.AttambaError("decoding keeps the L >= 1 most recent tokens; this layer has L = 0")
+        B, H, dh, N, D, L = self.B, self.H, self.dh, self.N, self.D, self.L
+        bf, i32 = torch.bfloat16, torch.int32
+        z = lambda *shape, dt=bf: torch.zeros(*shape, dtype=dt, device=device)  # noqa: E731
+        return A.Cache(z(2, B, N, D, dt=torch.float32), z(B, H, cap, dh), z(B, H, cap, dh), z(B, cap, dt=i32),
+                       z(B, H, L, dh), z(B, H, L, dh), z(B, dt=i32), z(B, dt=i32), self.P, self.offset)
+
+    def cache_from_prefill(self, cache, x, stream=None):
+        """Fill ``cache`` with what the last ``forward`` (over x, all n tokens of each sequence, uniform
+        chunks) leaves for decoding position n onwards: its chunk-end keys and values, its last L
+        tokens and the SSM states after token n - 1."""
+        B, n, H, dh = self.B, self.n, self.H, self.dh
+        pf = self.prefill
+        _, dt_k, dt_v, B_k, C_k, B_v, C_v = (t for t, _ in self.proj)
+        A.cache_from_prefill(cache, pf.K.view(B, n, H, dh), pf.V.view(B, n, H, dh), x, dt_k, dt_v, self.bias_k,
+                             self.bias_v, self.A_k, self.A_v, B_k, C_k, B_v, C_v, n, self.status, stream)
+
+    def decode_step(self, cache, x_t, stream=None):
+        """One new token per sequence under the inference mask M_test: x_t [B, D] bf16 -> y_t [B, D]
+        (the layer's own buffer).  The same seven projections as ``forward`` (one GEMM of B rows), the
+        decode step over ``cache`` (which it advances by one position), then W_O."""
+        B, H, dh, D = self.B, self.H, self.dh, self.D
+        bf = torch.bfloat16
+        if getattr(self, "_step", None) is None:
+            dev = self.W_in.device
+            self._step, c = [], 0
+            for (t, _) in self.proj:
+                self._step.append((torch.empty(B, t.shape[1], dtype=bf, device=dev), c))
+                c += t.shape[1]
+            self.o_t = torch.empty(B, H, dh, dtype=bf, device=dev)
+            self.y_t = torch.empty(B, D, dtype=bf, device=dev)
+            self._ws = {}
+        size = A.decode_workspace_size(cache)
+        if size not in self._ws:
+            self._ws[size] = torch.empty(size, dtype=torch.uint8, device=self.W_in.device)
+        q, dt_k, dt_v, B_k, C_k, B_v, C_v = (t for t, _ in self._step)
+        A.proj_gemm(x_t, self.W_in, self._step, self.status, stream)
+        A.decode_step(cache, q.view(B, H, dh), x_t, dt_k, dt_v, self.bias_k, self.bias_v, self.A_k, self.A_v, B_k,
+                      C_k, B_v, C_v, self.scale, self.o_t, self._ws[size], self.status, stream)
+        A.proj_gemm(self.o_t.view(B, H * dh), self.W_O, [(self.y_t, 0)], self.status, stream)
+        return self.y_t
+
+    @property
+    def step_projections(self):
+        """The last decode step's projections, named like ``projections``."""
+        return {k[2:]: t for k, (t, _) in zip(INPUT_PROJECTIONS, self._step)}
 
     def forward(self, x, cu_in=None, stream=None):
         """x [B n, D] bf16 -> y [B n, D] bf16 (the layer's own buffer)."""

@@ -15,7 +15,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import Guarded, assert_bf16_close, assert_written, f64, oracle_attention_seq
+from helpers import BF16_ATOL, Guarded, assert_bf16_close, assert_written, f64, oracle_attention_seq
 from oracle import chunks as OC
 from oracle import projection as OP
 from oracle import ssm as OS
@@ -122,3 +122,54 @@ def test_layer_stages_match_oracle(case):
     # 4. the output projection, from the GPU's O
     Ot = pf.O.view(T, H * DH).cpu()
     _gemm_check(y.cpu(), OP.project(f64(Ot), f64(w["W_O"])), Ot, w["W_O"], "y")
+
+
+@pytest.mark.parametrize("n0", [0, 120], ids=["from_empty_cache", "after_prefill_handoff"])
+def test_layer_decode_continues_its_prefill(n0):
+    """Decoding through the layer (Layer.decode_step) from an empty cache, or from the cache a
+    Layer.forward over the first n0 tokens leaves (Layer.cache_from_prefill): at every position t the
+    step's attention output is the M_test prefill row t of a Layer.forward over the whole sequence
+    (itself checked against the oracle above) within bf16 rounding, and the step's seven projections
+    and y_t match the oracle's products of the step's own inputs."""
+    B, steps, H, N, P, offset, L = 2, 40, 2, 16, 8, 3, 16
+    n = n0 + steps
+    D = H * DH
+    bf = torch.bfloat16
+    gen = torch.Generator().manual_seed(77 + n0)
+    s = 1.0 / math.sqrt(D)
+    shapes = {"W_Q": (H * DH, D), "W_dtK": (D, D), "W_dtV": (D, D), "W_BK": (N, D), "W_CK": (N, D),
+              "W_BV": (N, D), "W_CV": (N, D), "W_O": (D, H * DH)}
+    w = {k: (torch.randn(*shp, generator=gen) * s).to(bf) for k, shp in shapes.items()}
+    w["bias_k"], w["bias_v"] = W._dt_bias(D, gen), W._dt_bias(D, gen)
+    w["A_k"], w["A_v"] = W._A(D, N, gen), W._A(D, N, gen)
+    wg = {k: v.cuda() for k, v in w.items()}
+    x = torch.randn(B, n, D, generator=gen).to(bf)
+    scale = 1.0 / math.sqrt(DH)
+    args = (H, DH, N, wg, P, offset, L, A.MASK_TEST, scale)
+
+    full = layer.Layer(B, n, D, *args)
+    full.forward(x.view(B * n, D).cuda())
+    O_full = full.prefill.O.view(B, n, H, DH)
+    cap = n // P + 2
+    if n0 == 0:
+        dec = full
+        cache = dec.new_cache(cap)
+    else:
+        dec = layer.Layer(B, n0, D, *args)
+        xp = x[:, :n0].reshape(B * n0, D).contiguous().cuda()
+        dec.forward(xp)
+        cache = dec.new_cache(cap)
+        dec.cache_from_prefill(cache, xp)
+    for t in range(n0, n):
+        xt = x[:, t].contiguous()
+        y_t = dec.decode_step(cache, xt.cuda())
+        torch.cuda.synchronize()
+        err = (dec.o_t.float() - O_full[:, t].float()).abs().max().item()
+        assert err <= BF16_ATOL, f"o_t at position {t}: {err} from the prefill row"
+        sp = dec.step_projections
+        for name in layer.INPUT_PROJECTIONS:
+            _gemm_check(sp[name[2:]].cpu(), OP.project(f64(xt), f64(w[name])), xt, w[name], f"{name} at {t}")
+        ot = dec.o_t.view(B, H * DH).cpu()
+        _gemm_check(y_t.cpu(), OP.project(f64(ot), f64(w["W_O"])), ot, w["W_O"], f"y_t at {t}")
+    assert full.status.item() == 0 and dec.status.item() == 0
+    assert (cache.pos.cpu() == n).all()
