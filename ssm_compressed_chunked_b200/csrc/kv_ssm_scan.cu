@@ -289,8 +289,13 @@ __global__ void __launch_bounds__(kScanThreads, MINB) kv_ssm_scan_kernel(ScanArg
   // Software pipeline over token pairs: the deltas of the pair being computed
   // come from loads issued one pair earlier, and the loads for the pair after
   // next are issued once the registers they land in have been consumed.
+  // With one input per SSM (SPLIT_X) neither SSM's x is in L2 from the other's read, and the loads
+  // go a second pair further ahead (184-185 against 189 us on the bench shapes; with the shared
+  // input the deeper pipeline measured 2-3 us slower, so it stays one pair ahead there).
+  constexpr bool kAhead2 = SPLIT_X;
   float dlA[CPT], dxA[CPT], dlB[CPT], dxB[CPT];
   typename V::raw xA, zA, xB, zB;
+  typename V::raw xC = {}, zC = {}, xD = {}, zD = {};   // the pair after that (kAhead2)
   auto delta_of = [&](typename V::raw xr, typename V::raw zr, float (&dl)[CPT], float (&dx)[CPT]) {
     float xv[CPT], zv[CPT];
     V::unpack(xr, xv);
@@ -307,6 +312,10 @@ __global__ void __launch_bounds__(kScanThreads, MINB) kv_ssm_scan_kernel(ScanArg
     delta_of(V::load(x + tok(t_begin + 1) * D), V::load(dt + tok(t_begin + 1) * D), dlB, dxB);
     xA = V::load(x + tok(t_begin + 2) * D); zA = V::load(dt + tok(t_begin + 2) * D);
     xB = V::load(x + tok(t_begin + 3) * D); zB = V::load(dt + tok(t_begin + 3) * D);
+    if (kAhead2) {
+      xC = V::load(x + tok(t_begin + 4) * D); zC = V::load(dt + tok(t_begin + 4) * D);
+      xD = V::load(x + tok(t_begin + 5) * D); zD = V::load(dt + tok(t_begin + 5) * D);
+    }
   }
 
   auto step = [&](int t, const float* bc, const float (&dl)[CPT], const float (&dx)[CPT]) {
@@ -342,8 +351,14 @@ __global__ void __launch_bounds__(kScanThreads, MINB) kv_ssm_scan_kernel(ScanArg
       if (k + 1 < nt) step(t + 1, &sBC[k + 1][0], dlB, dxB);
       delta_of(xA, zA, dlA, dxA);
       delta_of(xB, zB, dlB, dxB);
-      xA = V::load(x + tok(t + 4) * D); zA = V::load(dt + tok(t + 4) * D);
-      xB = V::load(x + tok(t + 5) * D); zB = V::load(dt + tok(t + 5) * D);
+      if (kAhead2) {
+        xA = xC; zA = zC; xB = xD; zB = zD;
+        xC = V::load(x + tok(t + 6) * D); zC = V::load(dt + tok(t + 6) * D);
+        xD = V::load(x + tok(t + 7) * D); zD = V::load(dt + tok(t + 7) * D);
+      } else {
+        xA = V::load(x + tok(t + 4) * D); zA = V::load(dt + tok(t + 4) * D);
+        xB = V::load(x + tok(t + 5) * D); zB = V::load(dt + tok(t + 5) * D);
+      }
     }
   }
 }
