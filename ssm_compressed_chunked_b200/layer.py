@@ -86,7 +86,8 @@ class Layer:
     [out, in] layout (W_Q [H dh, D]; W_dtK, W_dtV [D, D]; W_BK ... W_CV [N, D];
     W_O [D, H dh]) and "bias_k", "bias_v" [D], "A_k", "A_v" [D, N] to fp32; all on
     the layer's device.  The chunking is uniform (P, offset) unless ``forward``
-    gets chunk offsets ``cu_in``; ``mode`` is MASK_TEST or MASK_TRAIN.
+    gets chunk offsets ``cu_in`` (then ``n_chunks`` must be their count);
+    ``mode`` is MASK_TEST or MASK_TRAIN.
 
     Decoding (pith.science review, "Core claim": the inference cache holds the
     chunk boundary states, and "If this is right": P = 8 with 64 leading tokens)
@@ -122,6 +123,7 @@ class Layer:
         self.prefill = Prefill(B, n, D, H, dh, N, n_chunks, bf, device=device, alloc=alloc)
         self.y = alloc((T, D), bf)
         self.status = self.prefill.status
+        self._step = None   # decode buffers, made by the first decode_step
 
     @property
     def projections(self):
@@ -129,11 +131,13 @@ class Layer:
         return {k[2:]: t for k, (t, _) in zip(INPUT_PROJECTIONS, self.proj)}
 
     # ---------------------------------------------------------------- decode (M_test, uniform chunks)
-    def new_cache(self, cap, device="cuda"):
+    def new_cache(self, cap, device=None):
         """An empty decode cache (every sequence at position 0) with room for ``cap`` chunk-end rows
-        per sequence and the layer's L most recent tokens, chunked like the layer (P, offset)."""
+        per sequence and the layer's L most recent tokens, chunked like the layer (P, offset); on the
+        layer's device unless ``device`` says otherwise."""
         if self.L < 1:
             raise A.AttambaError("decoding keeps the L >= 1 most recent tokens; this layer has L = 0")
+        device = self.W_in.device if device is None else device
         B, H, dh, N, D, L = self.B, self.H, self.dh, self.N, self.D, self.L
         bf, i32 = torch.bfloat16, torch.int32
         z = lambda *shape, dt=bf: torch.zeros(*shape, dtype=dt, device=device)  # noqa: E731
@@ -156,7 +160,7 @@ class Layer:
         decode step over ``cache`` (which it advances by one position), then W_O."""
         B, H, dh, D = self.B, self.H, self.dh, self.D
         bf = torch.bfloat16
-        if getattr(self, "_step", None) is None:
+        if self._step is None:
             dev = self.W_in.device
             self._step, c = [], 0
             for (t, _) in self.proj:
@@ -178,6 +182,8 @@ class Layer:
     @property
     def step_projections(self):
         """The last decode step's projections, named like ``projections``."""
+        if self._step is None:
+            raise A.AttambaError("no decode step has run on this layer")
         return {k[2:]: t for k, (t, _) in zip(INPUT_PROJECTIONS, self._step)}
 
     def forward(self, x, cu_in=None, stream=None):

@@ -141,3 +141,21 @@ def test_cache_bytes_covers_every_cache_array(B, H, N, L, cap):
     assert A.cache_bytes(0, H, dh, N, L, cap) == 0
     assert A.cache_bytes(B, H, dh, N, 0, cap) == 0
     assert A.cache_bytes(B, H, dh, N, L, 0) == 0
+
+
+def test_layer_rejects_weights_of_the_wrong_shape_or_type():
+    """layer.Layer checks every weight against the layer's sizes before it allocates anything."""
+    import torch
+    from ssm_compressed_chunked_b200 import layer
+    B, n, D, H, dh, N = 1, 16, 128, 2, 64, 16
+    bf = torch.bfloat16
+    shapes = {"W_Q": (H * dh, D), "W_dtK": (D, D), "W_dtV": (D, D), "W_BK": (N, D), "W_CK": (N, D),
+              "W_BV": (N, D), "W_CV": (N, D), "W_O": (D, H * dh)}
+    good = {k: torch.zeros(*s, dtype=bf) for k, s in shapes.items()}
+    for name in shapes:
+        for bad in (torch.zeros(shapes[name][0] + 8, shapes[name][1], dtype=bf),
+                    torch.zeros(*shapes[name], dtype=torch.float32)):
+            w = dict(good)
+            w[name] = bad
+            with pytest.raises(A.AttambaError, match=name):
+                layer.Layer(B, n, D, H, dh, N, w, 8, 0, 4, A.MASK_TEST, 0.125, device="cpu")
