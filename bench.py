@@ -631,7 +631,7 @@ def run_ours(args, ws, rank, local):
     if rank != 0:
         return
 
-    hbm, tf_burst, tf_sus, src = peaks()
+    hbm, tf_burst, _, src = peaks()
     mean = per.mean(axis=0)  # ms per launch: index, scan, attention
     kernels = {
         "chunk_index": {"ms": mean[0], "bytes": index_bytes},

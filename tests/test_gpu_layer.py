@@ -116,7 +116,7 @@ def test_layer_stages_match_oracle(case):
         q = f64(pr["Q"][rows]).reshape(n, H, DH)
         K = f64(pf.K[rows]).reshape(n, H, DH)
         V = f64(pf.V[rows]).reshape(n, H, DH)
-        ro, rl = oracle_attention_seq(q, K, V, np.asarray(starts[b]), n, L, mode, scale)
+        ro, _ = oracle_attention_seq(q, K, V, np.asarray(starts[b]), n, L, mode, scale)
         assert_bf16_close(f64(pf.O.view(T, H, DH)[rows]), ro, f"O of sequence {b}")
 
     # 4. the output projection, from the GPU's O
