@@ -28,6 +28,7 @@ SELECTION = [
     "tests/test_gpu_decode.py::test_decode_after_short_handoff_into_long_capacity",
     "tests/test_gpu_decode.py::test_full_cache_raises_status_bit",
     "tests/test_gpu_handoff.py",
+    "tests/test_gpu_layer.py",
 ]
 RUNNER = """
 import sys
