@@ -12,8 +12,10 @@ def _params(rng, D, N):
     return bias, A
 
 
-@pytest.mark.parametrize("P,offset,L", [(4, 0, 3), (4, 1, 1), (3, 2, 5), (8, 0, 9)])
+@pytest.mark.parametrize("P,offset,L", [(4, 0, 3), (4, 1, 1), (3, 2, 5), (8, 0, 9), (3, 1, 15), (4, 2, 20)])
 def test_decode_equals_test_mask_prefill(P, offset, L):
+    """A prefill of n0 = 11 tokens handed to the cache, then decoding to n = 20, reproduces the M_test
+    prefill rows (the last two cases keep a window longer than the prefill)."""
     rng = np.random.default_rng(P * 100 + offset * 10 + L)
     B, H, dh, N = 2, 2, 4, 5
     D = H * dh
