@@ -106,6 +106,7 @@ int32_t attamba_uniform_chunk_count(int32_t n, int32_t P, int32_t offset);
  *   cu_in    nullable [n_chunks+1] device: variable chunks (P, offset ignored);
  *            NULL: uniform chunks of size P with offset (offset mod P), and
  *            n_chunks must equal B * attamba_uniform_chunk_count(n, P, offset).
+ *   B, n     sequences and tokens per sequence; B * n < 2^31 (positions are int32).
  *   L        leading tokens, >= 0;  mode  ATTAMBA_MASK_TRAIN / _TEST.
  *   out      host struct of device arrays; out->n_chunks, ->B, ->n must match.
  *            out->cu receives the chunk starts (it may alias cu_in).
