@@ -41,6 +41,7 @@ def _gemm_check(Y, ref, X, Wm, what):
 # (B, n, H, N, chunking, L, mask): D = H * 64.  n = 300 leaves a partial 128-query tile; the
 # variable chunking passes chunk offsets to the layer instead of (P, offset)
 CASES = [
+    (1, 512, 16, 16, ("uniform", 8, 0), 64, "test"),   # the bench workload's width and mask, 512 tokens
     (2, 300, 2, 16, ("uniform", 8, 3), 16, "test"),
     (1, 257, 4, 32, ("uniform", 4, 0), 4, "train"),
     (2, 200, 2, 16, ("varlen", 2, 12), 8, "train"),
